@@ -1,0 +1,263 @@
+"""Paged KV pool, cache contents and decode attention (oracle).
+
+Test infrastructure only: imported by tests, the smoke check and the
+benchmark's CPU leg.  Nothing here is called by the library.
+
+What the pages define, and how this model reads it:
+
+* The cache is cut into fixed-size blocks of `block_size` token slots that
+  live anywhere in one physical pool; each sequence owns a block table
+  mapping logical block j to a physical block ("KV cache", The maths and
+  its paging paragraph; kv-cache-pagedattention-serving, PagedAttention:
+  virtual memory for GPUs).
+* Blocks are handed out only as a sequence grows, one free block per block
+  boundary crossed ("Managing the KV Cache", Answer Key item 2), and go
+  back to the free list once no sequence references them ("Managing the KV
+  Cache", Block Tables and Sharing).
+* Several sequences may reference the same immutable blocks through
+  reference counts; a fresh block is taken only when a sequence is about to
+  write into a tail block that others still share, and the shared block is
+  copied first (copy-on-write; "Managing the KV Cache", Block Tables and
+  Sharing; kv-cache-pagedattention-serving, The bonus: sharing via
+  copy-on-write).
+* Attention for a sequence runs over every cached token of that sequence
+  in logical order ("kv-cache-pagedattention-serving", PagedAttention:
+  virtual memory for GPUs).  This oracle deliberately gathers the blocks
+  into a contiguous buffer first, which is the plain definition the fused
+  kernel must reproduce.
+
+Readings where the pages are silent (each is listed in the design doc):
+
+* free list is FIFO: allocate from the head, release to the tail, in
+  logical-block order; its initial order is given by the caller;
+* a reservation that needs both a copy-on-write block and new blocks takes
+  the copy-on-write block first; the number of blocks needed is checked
+  before anything changes, so a failed reservation leaves no trace;
+* the copy-on-write copy covers the whole block for every layer, K and V;
+* a query of head i attends through KV head floor(i / G), G = H_q / H_kv;
+* no mask beyond the sequence length; the scale is a caller argument.
+"""
+from __future__ import annotations
+
+import collections
+import enum
+
+import numpy as np
+
+from . import fp8 as _fp8
+from .numerics import bits_to_f32, bits_to_f64
+
+
+class Status(enum.Enum):
+    OK = "ok"
+    INVALID_ARG = "invalid_arg"
+    NO_BLOCKS = "no_blocks"
+    NO_SEQ = "no_seq"
+    SEQ_EXISTS = "seq_exists"
+    SHARED_BLOCK = "shared_block"
+
+
+def _ceil_div(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+class PagedKVOracle:
+    """Block pool + cache contents + float64 attention.
+
+    Cache arrays use the pool layout [layer][block][kv_head][slot][head_dim]
+    and hold raw storage bits (uint16 for bf16 / fp16, uint8 codes for FP8).
+    `stored_layers` limits which layers keep contents (all by default), so
+    large workloads can be checked layer by layer.
+    """
+
+    def __init__(self, *, num_layers: int, num_kv_heads: int, head_dim: int, block_size: int,
+                 num_blocks: int, max_seqs: int, max_blocks_per_seq: int, kv_dtype: str,
+                 free_order=None, stored_layers=None):
+        self.L, self.H, self.d, self.B = num_layers, num_kv_heads, head_dim, block_size
+        self.num_blocks, self.max_seqs, self.mbps = num_blocks, max_seqs, max_blocks_per_seq
+        self.kv_dtype = kv_dtype
+        order = range(num_blocks) if free_order is None else [int(b) for b in free_order]
+        if sorted(order) != list(range(num_blocks)):
+            raise ValueError("free_order must be a permutation of the block ids")
+        self.free = collections.deque(order)
+        self.ref = [0] * num_blocks
+        self.tables: dict[int, list[int]] = {}
+        self.lens: dict[int, int] = {}
+        self.cow_log: list[tuple[int, int]] = []
+        layers = range(num_layers) if stored_layers is None else stored_layers
+        store = np.uint8 if kv_dtype == "fp8_e4m3" else np.uint16
+        shape = (num_blocks, num_kv_heads, block_size, head_dim)
+        self.k = {layer: np.zeros(shape, store) for layer in layers}
+        self.v = {layer: np.zeros(shape, store) for layer in layers}
+
+    # ------------------------------------------------------------------ pool
+    def reserve(self, seq: int, new_len: int) -> Status:
+        """Grow (or create) `seq` to hold `new_len` tokens."""
+        if not 0 <= seq < self.max_seqs or new_len < 0:
+            return Status.INVALID_ARG
+        table = self.tables.get(seq, [])
+        cur = self.lens.get(seq, 0)
+        if new_len < cur or _ceil_div(new_len, self.B) > self.mbps:
+            return Status.INVALID_ARG
+        cow = new_len > cur and cur % self.B != 0 and self.ref[table[-1]] > 1
+        grow = _ceil_div(new_len, self.B) - len(table)
+        if int(cow) + grow > len(self.free):
+            return Status.NO_BLOCKS
+        table = list(table)
+        if cow:
+            src = table[-1]
+            dst = self.free.popleft()
+            for layer in self.k:
+                self.k[layer][dst] = self.k[layer][src]
+                self.v[layer][dst] = self.v[layer][src]
+            self.ref[src] -= 1
+            self.ref[dst] = 1
+            table[-1] = dst
+            self.cow_log.append((src, dst))
+        for _ in range(grow):
+            b = self.free.popleft()
+            self.ref[b] = 1
+            table.append(b)
+        self.tables[seq] = table
+        self.lens[seq] = new_len
+        return Status.OK
+
+    def fork(self, parent: int, child: int) -> Status:
+        """`child` shares every block of `parent` (reference count + 1)."""
+        if not 0 <= child < self.max_seqs or not 0 <= parent < self.max_seqs:
+            return Status.INVALID_ARG
+        if parent not in self.tables:
+            return Status.NO_SEQ
+        if child in self.tables:
+            return Status.SEQ_EXISTS
+        self.tables[child] = list(self.tables[parent])
+        self.lens[child] = self.lens[parent]
+        for b in self.tables[child]:
+            self.ref[b] += 1
+        return Status.OK
+
+    def release(self, seq: int) -> Status:
+        """Drop `seq`; blocks whose count reaches zero return to the free tail."""
+        if seq not in self.tables:
+            return Status.NO_SEQ if 0 <= seq < self.max_seqs else Status.INVALID_ARG
+        for b in self.tables[seq]:
+            self.ref[b] -= 1
+            if self.ref[b] == 0:
+                self.free.append(b)
+        del self.tables[seq]
+        del self.lens[seq]
+        return Status.OK
+
+    def slot(self, seq: int, pos: int):
+        """(physical block, slot in block) for token `pos` of `seq`, or a Status."""
+        if seq not in self.tables:
+            return Status.NO_SEQ
+        if not 0 <= pos < self.lens[seq]:
+            return Status.INVALID_ARG
+        b = self.tables[seq][pos // self.B]
+        if self.ref[b] > 1:
+            return Status.SHARED_BLOCK
+        return b, pos % self.B
+
+    # ----------------------------------------------------------------- cache
+    def append(self, layer: int, seqs, positions, k_bits, v_bits, act_dtype: str,
+               k_inv=None, v_inv=None) -> Status:
+        """Write one K row and one V row per (seq, pos) into its cache slot.
+
+        `k_bits` / `v_bits`: [T, num_kv_heads, head_dim] activation bits.
+        For an FP8 pool the stored code is E4M3(fp32(x * inv_scale[layer, h])).
+        All targets are validated before anything is written.
+        """
+        slots = []
+        for s, p in zip(seqs, positions):
+            r = self.slot(int(s), int(p))
+            if isinstance(r, Status):
+                return r
+            slots.append(r)
+        if layer not in self.k:
+            return Status.OK
+        for t, (b, o) in enumerate(slots):
+            if self.kv_dtype == "fp8_e4m3":
+                xk = bits_to_f32(k_bits[t], act_dtype)
+                xv = bits_to_f32(v_bits[t], act_dtype)
+                self.k[layer][b, :, o, :] = _fp8.quantize(xk, np.asarray(k_inv[layer])[:, None])
+                self.v[layer][b, :, o, :] = _fp8.quantize(xv, np.asarray(v_inv[layer])[:, None])
+            else:
+                self.k[layer][b, :, o, :] = k_bits[t]
+                self.v[layer][b, :, o, :] = v_bits[t]
+        return Status.OK
+
+    def gather(self, layer: int, seq: int):
+        """Contiguous float64 K and V of `seq`: [len, num_kv_heads, head_dim].
+
+        FP8 values are decoded exactly; the per-head scale is applied by
+        `attention`.
+        """
+        n = self.lens[seq]
+        t = np.arange(n)
+        blocks = np.asarray(self.tables[seq], dtype=np.int64)[t // self.B]
+        kb = self.k[layer][blocks, :, t % self.B, :]
+        vb = self.v[layer][blocks, :, t % self.B, :]
+        if self.kv_dtype == "fp8_e4m3":
+            return _fp8.decode(kb), _fp8.decode(vb)
+        return bits_to_f64(kb, self.kv_dtype), bits_to_f64(vb, self.kv_dtype)
+
+    def attention(self, layer: int, seqs, q_bits, act_dtype: str, scale: float,
+                  k_scale=None, v_scale=None) -> np.ndarray:
+        """softmax(scale * q K^T) V per (sequence, query head), float64.
+
+        `q_bits`: [n, num_q_heads, head_dim] activation bits.  Query head i
+        uses KV head i // G.  Returns float64 [n, num_q_heads, head_dim].
+        """
+        q = bits_to_f64(q_bits, act_dtype)
+        n, hq, d = q.shape
+        group = hq // self.H
+        sc = float(np.float32(scale))
+        out = np.zeros((n, hq, d), np.float64)
+        for i, s in enumerate(seqs):
+            K, V = self.gather(layer, int(s))
+            for qh in range(hq):
+                h = qh // group
+                kh, vh = K[:, h, :], V[:, h, :]
+                if self.kv_dtype == "fp8_e4m3":
+                    kh = kh * float(k_scale[layer][h])
+                    vh = vh * float(v_scale[layer][h])
+                x = (kh @ q[i, qh]) * sc
+                p = np.exp(x - x.max())
+                p /= p.sum()
+                out[i, qh] = p @ vh
+        return out
+
+    # ------------------------------------------------------------ inspection
+    def table(self, seq: int) -> list[int]:
+        return list(self.tables[seq])
+
+    def free_list(self) -> list[int]:
+        return list(self.free)
+
+    def refcounts(self) -> list[int]:
+        return list(self.ref)
+
+    def check_invariants(self) -> None:
+        """Pool invariants the pages imply; raises AssertionError if broken.
+
+        * only a sequence's final block can be partly empty, so tail waste
+          is at most block_size - 1 ("Managing the KV Cache", Internal
+          Fragmentation);
+        * a block is on the free list iff nothing references it ("Managing
+          the KV Cache", Block Tables and Sharing);
+        * every block is either free or referenced, never both, never twice
+          on the free list; total references = total table entries.
+        """
+        counted = [0] * self.num_blocks
+        for seq, table in self.tables.items():
+            n = self.lens[seq]
+            assert len(table) == _ceil_div(n, self.B)
+            assert len(table) * self.B - n <= self.B - 1
+            for b in table:
+                counted[b] += 1
+        assert counted == self.ref
+        free = list(self.free)
+        assert len(set(free)) == len(free)
+        assert set(free) == {b for b in range(self.num_blocks) if self.ref[b] == 0}
+        assert len(free) + sum(1 for r in self.ref if r > 0) == self.num_blocks

@@ -1,0 +1,100 @@
+"""Planted mistakes in the oracle must be caught by its pins.
+
+Each case edits one line of an oracle function's source (a dropped term, a
+wrong index, a wrong rounding, a wrong list end), installs the edited
+function in place of the real one for the duration of the test, and runs
+the pin that should notice.  The pin must fail.
+"""
+import inspect
+import textwrap
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import fp8, paged, sizing
+
+import test_oracle_attention as att
+import test_oracle_fp8 as tf8
+import test_oracle_pool as pool
+import test_oracle_sizing as tsz
+
+
+def _mutated(func, old, new):
+    src = textwrap.dedent(inspect.getsource(func))
+    assert src.count(old) == 1, f"mutation anchor not unique in {func.__name__}: {old!r}"
+    src = src.replace(old, new)
+    ns = dict(func.__globals__)
+    exec(compile(src, f"<mutant {func.__name__}>", "exec"), ns)
+    return ns[func.__name__]
+
+
+MUTANTS = [
+    # (target object, attribute, old text, new text, pin to run)
+    (fp8, "encode_f32", "np.rint(", "np.floor(",
+     lambda: tf8.test_encode_brute_force_random_fp32()),
+    (fp8, "encode_f32", "e = np.maximum(ex - 1, -6)", "e = np.maximum(ex - 1, -7)",
+     lambda: tf8.test_encode_matches_brute_force_all_bf16()),
+    (fp8, "decode", "(8 + m) * np.exp2(e.astype(np.float64) - 10.0)", "(8 + m) * np.exp2(e.astype(np.float64) - 9.0)",
+     lambda: tf8.test_code_values_from_definition()),
+    (sizing, "kv_bytes_per_token", "return 2 * layers", "return layers",
+     None),
+    (sizing, "pool_blocks", "budget_bytes // (bytes_per_token * block_size)",
+     "budget_bytes // bytes_per_token // block_size + 1", None),
+    (paged.PagedKVOracle, "attention", "h = qh // group", "h = qh % self.H",
+     lambda: att.test_matches_scalar_brute_force(2)),
+    (paged.PagedKVOracle, "attention", "x = (kh @ q[i, qh]) * sc", "x = (kh @ q[i, qh])",
+     lambda: att.test_matches_scalar_brute_force(1)),
+    (paged.PagedKVOracle, "attention", "kh, vh = K[:, h, :], V[:, h, :]", "kh, vh = K[:, h, :], K[:, h, :]",
+     lambda: att.test_matches_torch_sdpa_float64()),
+    (paged.PagedKVOracle, "attention", "vh = vh * float(v_scale[layer][h])", "vh = vh * float(k_scale[layer][h])",
+     lambda: att.test_fp8_matches_scalar_brute_force()),
+    (paged.PagedKVOracle, "gather", "blocks = np.asarray(self.tables[seq], dtype=np.int64)[t // self.B]",
+     "blocks = np.asarray(self.tables[seq], dtype=np.int64)[t % len(self.tables[seq])]",
+     lambda: att.test_matches_scalar_brute_force(1)),
+    (paged.PagedKVOracle, "reserve", "cow = new_len > cur and cur % self.B != 0 and self.ref[table[-1]] > 1",
+     "cow = False", lambda: pool.test_parallel_sampling_cow_seven_copies_one_in_place()),
+    (paged.PagedKVOracle, "reserve", "if int(cow) + grow > len(self.free):", "if grow > len(self.free):",
+     lambda: pool.test_cow_and_growth_need_is_checked_before_any_change()),
+    (paged.PagedKVOracle, "release", "self.free.append(b)", "self.free.appendleft(b)",
+     lambda: pool.test_release_returns_blocks_in_logical_order_once_unreferenced()),
+    (paged.PagedKVOracle, "slot", "if self.ref[b] > 1:", "if self.ref[b] > 2:",
+     lambda: pool.test_invalid_calls()),
+    (paged.PagedKVOracle, "append", "self.k[layer][b, :, o, :] = k_bits[t]", "self.k[layer][b, :, o - 1, :] = k_bits[t]",
+     lambda: pool.test_append_writes_the_slot_and_nothing_else()),
+]
+
+
+def _sizing_pins(golden_dir):
+    import json
+    import os
+    with open(os.path.join(golden_dir, "printed_sizing.json")) as f:
+        printed = json.load(f)
+    tsz.test_bytes_per_token_printed(printed)
+    tsz.test_capacity_12gib(printed)
+
+
+@pytest.mark.parametrize("case", range(len(MUTANTS)))
+def test_planted_mistake_is_caught(case, monkeypatch, golden_dir):
+    target, name, old, new, pin = MUTANTS[case]
+    real = getattr(target, name)
+    func = real if inspect.isfunction(real) else real.__func__
+    monkeypatch.setattr(target, name, _mutated(func, old, new))
+    if target is sizing:
+        # sizing helpers call each other through module globals, so the
+        # capacity pins see the mutant too
+        with pytest.raises(AssertionError):
+            _sizing_pins(golden_dir)
+        return
+    # an assertion, or the mutant crashing on a state the real code never reaches
+    with pytest.raises((AssertionError, IndexError)):
+        pin()
+
+
+def test_unmutated_pins_pass(golden_dir):
+    _sizing_pins(golden_dir)
+    tf8.test_code_values_from_definition()
+    att.test_matches_scalar_brute_force(2)
+    pool.test_invalid_calls()
+    assert oracle.PagedKVOracle is paged.PagedKVOracle
+    assert np.isfinite(fp8.decode(np.arange(0x7F, dtype=np.uint8))).all()
