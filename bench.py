@@ -1,0 +1,581 @@
+"""Benchmark of the paged decode-attention hot path on B200.
+
+One step = one decode step of the workload: reserve one more slot per
+sequence (block manager; a block on boundary crossings, copy-on-write where
+a shared tail is written), then for every layer append the step's K/V row
+per sequence and run decode attention for every sequence -- all through the
+C ABI (libpa.so).  Default workload: the 8B-class GQA layer (64 sequences,
+lengths uniform in [128, 4096], 32 query / 8 KV heads, head_dim 128, bf16,
+16-token blocks, shuffled pool sized 1.25x the need at the end of the run).
+
+Metric: achieved HBM GB/s of the step's algorithmic bytes (KV read by the
+decode + Q + O + block-table entries + appended rows read and written),
+with its fraction of the measured B200 copy bandwidth, and decode tokens/s
+(sequences x steps / time).  Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Under torchrun each rank runs its own replica of the workload on its own GPU
+(the path has no exchange step: replicas only, weak scaling); the timed
+region is bracketed by a barrier and synchronize, and the time is the max
+over ranks.  `--impl reference` times the CPU oracle (float64 NumPy) on the
+host cores instead, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attn: achieved HBM GB/s (% of B200 peak), decode tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gqa8b",
+                    choices=["tiny", "gqa8b", "gqa70b_headroom", "mha7b_share", "fp8_long"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--partition", type=int, default=None,
+                    help="partition_tokens for decode (default: the workload's)")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
+
+
+def describe(w, partition):
+    return {
+        "workload": f"{w.name}: {len(w.seq_ids)} seqs, {w.num_layers} layer(s), "
+                    f"{w.num_q_heads} q / {w.num_kv_heads} KV heads, d{w.head_dim}, "
+                    f"{w.kv_dtype} KV, block {w.block_size}",
+        "seqs": len(w.seq_ids),
+        "layers": w.num_layers,
+        "q_heads": w.num_q_heads,
+        "kv_heads": w.num_kv_heads,
+        "head_dim": w.head_dim,
+        "block_size": w.block_size,
+        "kv_dtype": w.kv_dtype,
+        "pool_blocks": w.num_blocks,
+        "partition_tokens": partition,
+        "l2": "inputs larger than L2 (KV working set >> 126 MB); no flush",
+    }
+
+
+def step_bytes(w, lens_before):
+    """Algorithmic HBM bytes of one step (all layers), and of its decode alone.
+
+    decode: every cached token's K and V row once per (seq, KV head) + Q + O +
+    one block-table entry per block; append: new K/V rows read + written.
+    Shared blocks (parallel sampling) are counted once (distinct bytes).
+    """
+    kvb = 1 if w.kv_dtype == "fp8_e4m3" else 2
+    n = len(w.seq_ids)
+    row = 2 * w.num_kv_heads * w.head_dim * kvb           # K and V of one token, one layer
+    tokens = sum(lens_before[s] + 1 for s in w.seq_ids)
+    if w.forks:
+        # distinct tokens: shared prompt blocks once per family
+        fam = {}
+        for parent, child in w.forks:
+            fam.setdefault(parent, []).append(child)
+        shared_full = 0
+        for parent in fam:
+            shared_full += (w.prefill_lens[parent] // w.block_size) * w.block_size * len(fam[parent])
+        tokens -= shared_full
+    blocks = sum(math.ceil((lens_before[s] + 1) / w.block_size) for s in w.seq_ids)
+    qo = 2 * n * w.num_q_heads * w.head_dim * 2
+    decode = tokens * row + qo + 4 * blocks
+    append = n * 2 * w.num_kv_heads * w.head_dim * (2 + kvb)
+    return w.num_layers * (decode + append), w.num_layers * decode
+
+
+def logical_decode_bytes(w, lens_before):
+    kvb = 1 if w.kv_dtype == "fp8_e4m3" else 2
+    row = 2 * w.num_kv_heads * w.head_dim * kvb
+    return w.num_layers * sum((lens_before[s] + 1) * row for s in w.seq_ids)
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception:
+            self._nvml = None
+        return self
+
+    def _run(self):
+        nv = self._nvml
+        names = {
+            0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+            0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, nm in names.items():
+                    if r & bit:
+                        self.reasons.add(nm)
+            except Exception:
+                break
+            time.sleep(0.002)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        return {
+            "sm_mhz": statistics.median(self.samples) if self.samples else None,
+            "sm_max_mhz": self.max_mhz,
+            "reasons": sorted(self.reasons),
+            "samples": len(self.samples),
+        }
+
+
+def traffic_record(kernel_key):
+    """ncu DRAM bytes per decode launch, if recorded for this exact kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    r = rec.get(kernel_key)
+    if not r or r.get("source_sha") != source_sha():
+        return None
+    return r
+
+
+def source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "pagedattention_decode_03_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+# ======================================================================== ours
+class Runner:
+    """Pool + per-step inputs for one replica, driven through the C ABI."""
+
+    def __init__(self, w, device, partition, seed):
+        import torch
+        import pagedattention_decode_03_b200 as pa
+        self.torch, self.pa, self.w = torch, pa, w
+        self.dev = device
+        self.partition = partition
+        gen = torch.Generator(device=device)
+        gen.manual_seed(1000 + seed)
+        act = torch.bfloat16 if w.act_dtype == "bf16" else torch.float16
+        self.act = act
+        L, H, Hq, d = w.num_layers, w.num_kv_heads, w.num_q_heads, w.head_dim
+        kw = {}
+        if w.kv_dtype == "fp8_e4m3":
+            # calibration: amax/448 of N(0,1) data per (layer, head), computed on the
+            # prefill the replica writes (see prefill below)
+            self.amax = torch.zeros((L, H), dtype=torch.float32, device=device)
+        self.scales = None
+        # prefill data per (layer, seq) generated on the device
+        self.prefill_data = {}
+        for layer in range(L):
+            for s, n in w.prefill_lens.items():
+                k = torch.randn((n, H, d), generator=gen, device=device, dtype=torch.float32).to(act)
+                v = torch.randn((n, H, d), generator=gen, device=device, dtype=torch.float32).to(act)
+                self.prefill_data[(layer, s)] = (k, v)
+                if w.kv_dtype == "fp8_e4m3":
+                    self.amax[layer] = torch.maximum(self.amax[layer], torch.maximum(
+                        k.float().abs().amax(dim=(0, 2)), v.float().abs().amax(dim=(0, 2))))
+        if w.kv_dtype == "fp8_e4m3":
+            ks = (self.amax * 1.02 / 448.0).float().contiguous()
+            inv = (1.0 / ks).float().contiguous()
+            self.scales = (ks, ks.clone(), inv, inv.clone())
+            kw = dict(k_scale=self.scales[0], v_scale=self.scales[1],
+                      k_inv_scale=self.scales[2], v_inv_scale=self.scales[3])
+        order = w.free_order()
+        self.pool = pa.pa_pool_create(
+            num_layers=L, num_kv_heads=H, block_size=w.block_size, num_blocks=w.num_blocks,
+            max_seqs=w.max_seqs, max_blocks_per_seq=w.max_blocks_per_seq, kv_dtype=w.kv_dtype,
+            act_dtype=w.act_dtype, free_order=order, device=device,
+            min_partition_tokens=min(512, partition) if partition and partition > 0 else 0, **kw)
+        for s in sorted(w.prefill_lens):
+            n = w.prefill_lens[s]
+            pa.pa_alloc_blocks(self.pool, s, n)
+            for layer in range(L):
+                k, v = self.prefill_data.pop((layer, s))
+                pa.pa_append_kv(self.pool, layer, [s] * n, list(range(n)), k, v)
+        for parent, child in w.forks:
+            pa.pa_fork_cow(self.pool, parent, child)
+        torch.cuda.synchronize(device)
+        # per-step inputs: a few distinct sets, cycled
+        n = len(w.seq_ids)
+        self.nsets = 4
+        self.q = [torch.randn((L, n, Hq, d), generator=gen, device=device).to(act) for _ in range(self.nsets)]
+        self.kn = [torch.randn((L, n, H, d), generator=gen, device=device).to(act) for _ in range(self.nsets)]
+        self.vn = [torch.randn((L, n, H, d), generator=gen, device=device).to(act) for _ in range(self.nsets)]
+        self.out = torch.empty((L, n, Hq, d), dtype=act, device=device)
+        self.seqs = np.asarray(w.seq_ids, np.int32)
+        self.lens = np.asarray([w.lens_before_step(0)[s] for s in w.seq_ids], np.int32)
+        self.step_idx = 0
+        self.L = pa.lib()
+        self.i32p = ctypes.POINTER(ctypes.c_int32)
+
+    def lens_dict(self):
+        return {s: int(n) for s, n in zip(self.w.seq_ids, self.lens)}
+
+    def step(self, stream, q=None, kn=None, vn=None, out=None, dec_events=None):
+        """One decode step through the C ABI (host arrays prebuilt)."""
+        w, L = self.w, self.L
+        k = self.step_idx % self.nsets
+        q = self.q[k] if q is None else q
+        kn = self.kn[k] if kn is None else kn
+        vn = self.vn[k] if vn is None else vn
+        out = self.out if out is None else out
+        n = len(self.seqs)
+        new = self.lens + 1
+        done = ctypes.c_int32()
+        sp = self.seqs.ctypes.data_as(self.i32p)
+        st = L.pa_alloc_blocks_n(self.pool.handle, n, sp, new.ctypes.data_as(self.i32p), stream,
+                                 ctypes.byref(done))
+        if st != 0:
+            raise RuntimeError(f"pa_alloc_blocks_n: {self.pa.pa_last_error()}")
+        pos = self.lens.ctypes.data_as(self.i32p)
+        for layer in range(w.num_layers):
+            st = L.pa_append_kv(self.pool.handle, layer, n, sp, pos, ctypes.c_void_p(kn[layer].data_ptr()),
+                                ctypes.c_void_p(vn[layer].data_ptr()), stream)
+            if st != 0:
+                raise RuntimeError(f"pa_append_kv: {self.pa.pa_last_error()}")
+            if dec_events is not None:
+                dec_events[0].record()
+            st = L.pa_decode_attention(self.pool.handle, layer, n, sp, w.num_q_heads,
+                                       ctypes.c_void_p(q[layer].data_ptr()),
+                                       ctypes.c_void_p(out[layer].data_ptr()), ctypes.c_float(w.scale),
+                                       self.partition, stream)
+            if dec_events is not None:
+                dec_events[1].record()
+                dec_events = None  # time the first layer's decode only
+            if st != 0:
+                raise RuntimeError(f"pa_decode_attention: {self.pa.pa_last_error()}")
+        self.lens = new
+        self.step_idx += 1
+
+
+def run_ours(a, rank, world, local_rank):
+    import torch
+    import workloads
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    from pagedattention_decode_03_b200 import build as _b
+    if rank == 0 or world == 1:
+        _b.build()
+    if world > 1:
+        torch.distributed.barrier()
+    total_steps = a.warmup + a.steps + (0 if a.no_e2e else a.warmup + a.steps)
+    w = workloads.workload(a.workload, seed=a.seed + rank, steps=total_steps)
+    partition = w.partition_tokens if a.partition is None else a.partition
+    r = Runner(w, device, partition, a.seed + rank)
+    stream_obj = torch.cuda.current_stream(device)
+    stream = ctypes.c_void_p(stream_obj.cuda_stream)
+    pa = r.pa
+
+    for _ in range(a.warmup):
+        r.step(stream)
+    torch.cuda.synchronize(device)
+
+    lens0 = r.lens_dict()
+    bytes_step = [step_bytes(w, {s: lens0[s] + i for s in lens0}) for i in range(a.steps)]
+    total_bytes = sum(b for b, _ in bytes_step)
+    dec_bytes = [d for _, d in bytes_step]
+    logical = sum(logical_decode_bytes(w, {s: lens0[s] + i for s in lens0}) for i in range(a.steps))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = pa.pa_launch_count(r.pool)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index) as clk:
+        start.record()
+        for i in range(a.steps):
+            r.step(stream, dec_events=ev[i])
+        end.record()
+        torch.cuda.synchronize(device)
+    launches = pa.pa_launch_count(r.pool) - launches0
+    ms = start.elapsed_time(end)
+    dec_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+    bits = pa.pa_check_device_errors(r.pool)
+    if bits:
+        raise RuntimeError(f"device error bits 0x{bits:x}")
+    tmax = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(tmax, op=torch.distributed.ReduceOp.MAX)
+    ms = float(tmax.item())
+
+    # ---- end to end: host (pinned) inputs in, output back, every step
+    e2e = None
+    if not a.no_e2e:
+        n = len(w.seq_ids)
+        hq = torch.empty_like(r.q[0], device="cpu").pin_memory()
+        hk = torch.empty_like(r.kn[0], device="cpu").pin_memory()
+        hv = torch.empty_like(r.vn[0], device="cpu").pin_memory()
+        ho = torch.empty_like(r.out, device="cpu").pin_memory()
+        hq.copy_(r.q[0].cpu()); hk.copy_(r.kn[0].cpu()); hv.copy_(r.vn[0].cpu())
+        dq, dk, dv = torch.empty_like(r.q[0]), torch.empty_like(r.kn[0]), torch.empty_like(r.vn[0])
+        for _ in range(a.warmup):
+            dq.copy_(hq, non_blocking=True); dk.copy_(hk, non_blocking=True); dv.copy_(hv, non_blocking=True)
+            r.step(stream, dq, dk, dv, r.out)
+            ho.copy_(r.out, non_blocking=True)
+        torch.cuda.synchronize(device)
+        lens1 = r.lens_dict()
+        e2e_bytes = sum(step_bytes(w, {s: lens1[s] + i for s in lens1})[0] for i in range(a.steps))
+        if world > 1:
+            torch.distributed.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(device)
+        s0.record()
+        for i in range(a.steps):
+            dq.copy_(hq, non_blocking=True); dk.copy_(hk, non_blocking=True); dv.copy_(hv, non_blocking=True)
+            r.step(stream, dq, dk, dv, r.out)
+            ho.copy_(r.out, non_blocking=True)
+        s1.record()
+        torch.cuda.synchronize(device)
+        e_ms = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device=device)
+        if world > 1:
+            torch.distributed.all_reduce(e_ms, op=torch.distributed.ReduceOp.MAX)
+        e_ms = float(e_ms.item())
+        e2e = {"value": world * e2e_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel()) * 2,
+               "d2h_bytes_per_step": ho.numel() * 2, "ms_per_step": e_ms / a.steps}
+
+    peak, peak_src = peaks()
+    value = world * total_bytes / (ms * 1e-3) / 1e9
+    dec_mean = statistics.mean(dec_ms)
+    achieved = statistics.mean(dec_bytes) / w.num_layers / (dec_mean * 1e-3) / 1e9
+    tr = traffic_record(f"{w.name}:decode")
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "pct_of_peak": round(100 * value / world / peak, 1),
+        "decode_tokens_per_s": round(world * len(w.seq_ids) * a.steps / (ms * 1e-3), 1),
+        "n_gpus": world,
+        "steps": a.steps,
+        "warmup": a.warmup,
+        "ms_per_step": round(ms / a.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.kv_dtype if w.kv_dtype != "fp8_e4m3" else "fp8_e4m3 KV / bf16 act",
+        "data": "synthetic (seeded N(0,1) K/V/Q, seeded lengths and block placement)",
+        "config": {**describe(w, partition), "parallelism": f"replicas x{world} (no exchange step)"},
+        "roofline": {
+            "kernel": "decode attention (decode kernel + split-KV reduce), first layer of each step",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_source": peak_src,
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": tr["dram_bytes_per_launch"] if tr else None,
+            "algorithmic_bytes_per_launch": int(statistics.mean(dec_bytes) / w.num_layers),
+            "launch_ms": round(dec_mean, 5),
+        },
+        "logical_decode_gbs": round(world * logical / (ms * 1e-3) / 1e9, 1),
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    if rank == 0 and not a.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(w, a.cpu_seconds, lens0)
+    return line
+
+
+# ==================================================================== oracle
+def _oracle_setup(w, lens_before, seqs):
+    """Oracle pool holding the sample sequences at `lens_before`."""
+    from oracle import PagedKVOracle
+    from workloads import prefill_kv_bits, step_kv_bits
+    order = w.free_order()
+    o = PagedKVOracle(num_layers=w.num_layers, num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
+                      block_size=w.block_size, num_blocks=w.num_blocks, max_seqs=w.max_seqs,
+                      max_blocks_per_seq=w.max_blocks_per_seq, kv_dtype=w.kv_dtype,
+                      free_order=order, stored_layers=[0])
+    ki = vi = None
+    if w.kv_dtype == "fp8_e4m3":
+        from workloads import fp8_scales
+        sc = fp8_scales(w, 0)
+        ki, vi = sc[2], sc[3]
+        o._scales = sc
+    for s in seqs:
+        n = w.prefill_lens.get(s, lens_before[s])
+        o.reserve(s, n)
+        k, v = prefill_kv_bits(w, 0, s, n)
+        o.append(0, [s] * n, list(range(n)), k, v, w.act_dtype, ki, vi)
+    return o
+
+
+class OracleSample:
+    """The oracle holding a bounded sample of the workload: the first (up to)
+    16 sequences, layer 0.  One step = reserve + append + float64 attention
+    for those sequences, as the GPU step does for all of them."""
+
+    def __init__(self, w, lens_before):
+        seqs = list(w.seq_ids)[: max(1, min(len(w.seq_ids), 16))]
+        if w.forks:
+            seqs = [s for s in seqs if s in w.prefill_lens][:4]
+        self.w, self.seqs = w, seqs
+        self.o = _oracle_setup(w, lens_before, seqs)
+        self.lens = {s: self.o.lens[s] for s in seqs}
+        self.idx = [w.seq_ids.index(s) for s in seqs]
+        self.sub = _subset(w, seqs)
+        self.k = 0
+
+    def step(self):
+        from workloads import step_kv_bits, step_q_bits
+        w, o, seqs = self.w, self.o, self.seqs
+        ki = vi = ks = vs = None
+        if w.kv_dtype == "fp8_e4m3":
+            ks, vs, ki, vi = o._scales
+        for s in seqs:
+            o.reserve(s, self.lens[s] + 1)
+        k, v = step_kv_bits(w, self.k, 0)
+        o.append(0, seqs, [self.lens[s] for s in seqs], k[self.idx], v[self.idx], w.act_dtype, ki, vi)
+        q = step_q_bits(w, self.k, 0)[self.idx]
+        o.attention(0, seqs, q, w.act_dtype, w.scale, ks, vs)
+        nbytes = step_bytes(self.sub, self.lens)[0] / w.num_layers
+        for s in seqs:
+            self.lens[s] += 1
+        self.k += 1
+        return nbytes
+
+
+def _threads():
+    from threadpoolctl import threadpool_info
+    return max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+
+
+def cpu_baseline(w, seconds, lens_before, kind="oracle"):
+    """Time the float64 oracle on the host cores on a bounded sample."""
+    smp = OracleSample(w, lens_before)
+    t0 = time.perf_counter()
+    steps = 0
+    nbytes = 0.0
+    while (time.perf_counter() - t0 < seconds and steps < 200) or steps == 0:
+        nbytes += smp.step()
+        steps += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": _threads(),
+            "host_cpus": os.cpu_count(), "kind": kind,
+            "sample": f"{steps} decode step(s) of layer 0 for {len(smp.seqs)} of {len(w.seq_ids)} "
+                      f"sequences (reserve + append + float64 attention), {dt:.1f} s"}
+
+
+def _subset(w, seqs):
+    import dataclasses
+    return dataclasses.replace(w, seq_ids=tuple(seqs), forks=(),
+                               prefill_lens={s: w.prefill_lens.get(s, 0) for s in seqs})
+
+
+def run_reference(a):
+    import workloads
+    w = workloads.workload(a.workload, seed=a.seed, steps=a.warmup + a.steps)
+    partition = w.partition_tokens if a.partition is None else a.partition
+    lens0 = w.lens_before_step(0)
+    smp = OracleSample(w, lens0)
+    for _ in range(a.warmup):
+        smp.step()
+    nbytes = 0.0
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        nbytes += smp.step()
+    dt = time.perf_counter() - t0
+    value = round(nbytes / dt / 1e9, 4)
+    sample = (f"each step: one decode step of layer 0 for {len(smp.seqs)} of {len(w.seq_ids)} "
+              f"sequences (reserve + append + float64 attention)")
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": a.gpus, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": round(1000 * dt / a.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded N(0,1) K/V/Q, seeded lengths and block placement)",
+        "config": {**describe(w, partition), "parallelism": "host cores"},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": _threads(), "host_cpus": os.cpu_count(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def main():
+    a = parse()
+    if a.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if a.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(a)), flush=True)
+        return
+    import torch
+    import datetime
+    if world > 1:
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=120),
+            device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(a, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,227 @@
+/*
+ * pa.h -- C ABI of the paged decode-attention library (libpa.so).
+ *
+ * The library implements single-query decode attention over a paged KV
+ * cache on one NVIDIA B200 (sm_100a), plus the pieces that keep the cache:
+ * a host-side block manager (free list, per-sequence block tables,
+ * reference counts, copy-on-write of a shared tail block) and the kernel
+ * that writes each step's new K/V rows into their cache slots.
+ *
+ * What the operations compute is fixed by three public pages:
+ *   [KVC] "KV cache" (AI engineering visualised): The maths, and the
+ *         paragraph on paged attention (block tables, blocks handed out as
+ *         a sequence grows, waste bounded by one block);
+ *   [MKV] "Managing the KV Cache": Reproduce Bytes per Token, Internal
+ *         Fragmentation, Block Tables and Sharing, Quantized KV, Answer Key;
+ *   [PAS] "kv-cache-pagedattention-serving": PagedAttention: virtual memory
+ *         for GPUs; The bonus: sharing via copy-on-write.
+ *
+ * Conventions for every call:
+ *   - Every call returns a pa_status.  Out-parameters are written only when
+ *     the call returns PA_OK.
+ *   - A call that fails on the host leaves the pool exactly as it was; in
+ *     particular PA_ERR_NO_BLOCKS is detected before anything changes.
+ *   - Device work is enqueued on the caller's stream and never waited for,
+ *     except by pa_check_device_errors.  `stream` is a cudaStream_t passed
+ *     as void*; NULL means the legacy default stream.  The pool's device
+ *     metadata is updated in stream order: calls on one pool that use
+ *     different streams must be ordered by the caller.
+ *   - The caller owns every device buffer (caches, scales, workspace,
+ *     q / out / k_new / v_new) and keeps it alive while work that uses it is
+ *     in flight.  The pool owns only host memory.
+ *   - A pool is not thread-safe; use one pool per host thread or lock.
+ *   - Sequence ids are integers in [0, max_seqs).
+ *   - pa_last_error() returns a description of the last failure on the
+ *     calling thread.
+ *
+ * Device data layout (bytes, row-major, caller-allocated):
+ *   k_cache, v_cache: [num_layers][num_blocks][num_kv_heads][block_size][head_dim]
+ *       elements of kv_dtype.  One (layer, block, kv_head) tile is one
+ *       contiguous block_size x head_dim slab.  A physical block id names
+ *       the same tile position in every layer, so one block holds
+ *       block_size token slots of the whole per-token footprint
+ *       2 x layers x kv_heads x head_dim x bytes ([MKV] Reproduce Bytes per
+ *       Token).  Base addresses must be 16-byte aligned.
+ *   q, out:           [n][num_q_heads][head_dim] act_dtype.
+ *   k_new, v_new:     [T][num_kv_heads][head_dim] act_dtype.
+ *   k_scale, v_scale, k_inv_scale, v_inv_scale: [num_layers][num_kv_heads] fp32
+ *       (FP8 pools only).
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct pa_pool pa_pool;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = -1,  /* bad argument, shape, pointer or sequence id */
+  PA_ERR_NO_BLOCKS = -2,    /* the free list cannot cover the reservation */
+  PA_ERR_NO_SEQ = -3,       /* the sequence does not exist */
+  PA_ERR_SEQ_EXISTS = -4,   /* fork target already exists */
+  PA_ERR_SHARED_BLOCK = -5, /* append into a block other sequences share */
+  PA_ERR_CUDA = -6,         /* a CUDA runtime call failed */
+  PA_ERR_DEVICE_CHECK = -7  /* a kernel's own bounds/timeout check fired */
+} pa_status;
+
+typedef enum {
+  PA_BF16 = 0,
+  PA_FP16 = 1,
+  PA_FP8_E4M3 = 2 /* OCP FP8 E4M3, KV storage only */
+} pa_dtype;
+
+/* Bits of the device error word read by pa_check_device_errors. */
+#define PA_DEVERR_BAD_BLOCK 0x1u   /* a table entry outside [0, num_blocks) */
+#define PA_DEVERR_BAD_LEN 0x2u     /* a sequence length beyond its table */
+#define PA_DEVERR_TIMEOUT 0x4u     /* a bounded wait on a copy gave up */
+
+typedef struct {
+  int32_t num_layers;
+  int32_t num_kv_heads;
+  int32_t head_dim;           /* must be 128 */
+  int32_t block_size;         /* tokens per block: 16 (32 accepted by the block manager only) */
+  int32_t num_blocks;         /* physical blocks in the pool */
+  int32_t max_seqs;           /* sequence ids are 0 .. max_seqs-1 */
+  int32_t max_blocks_per_seq; /* block-table capacity of one sequence */
+  int32_t kv_dtype;           /* pa_dtype of the cache */
+  int32_t act_dtype;          /* pa_dtype of q, out, k_new, v_new: PA_BF16 or PA_FP16;
+                                 equal to kv_dtype unless kv_dtype is PA_FP8_E4M3 */
+  int32_t min_partition_tokens; /* smallest fixed split-KV partition a decode call may ask
+                                   for (sizes the workspace); 0 selects 512 */
+  void *k_cache;              /* device, caller-owned; NULL together with v_cache makes a
+                                 host-only pool (block manager only, no device calls) */
+  void *v_cache;
+  const float *k_scale;       /* device fp32 [L][H_kv]: K dequantisation scale (FP8 only) */
+  const float *v_scale;       /* device fp32 [L][H_kv]: V dequantisation scale (FP8 only) */
+  const float *k_inv_scale;   /* device fp32 [L][H_kv]: fp32(1/k_scale), used to quantise */
+  const float *v_inv_scale;   /* device fp32 [L][H_kv]: fp32(1/v_scale) */
+  void *workspace;            /* device, caller-owned, >= pa_workspace_size(desc) bytes,
+                                 256-byte aligned; contents need no initialisation */
+  size_t workspace_bytes;
+  const int32_t *free_order;  /* host, optional: initial free-list order, a permutation
+                                 of 0..num_blocks-1 (copied); NULL = ascending */
+  int32_t device;             /* CUDA device ordinal holding the buffers */
+} pa_pool_desc;
+
+/* Bytes of device workspace a pool with this description needs: the
+ * device mirror of the block tables and lengths, the split-KV partial
+ * results and an error word.  Pure arithmetic; needs no GPU. */
+size_t pa_workspace_size(const pa_pool_desc *desc);
+
+/* Validate `desc` and create the host state of a pool.  Needs no GPU and
+ * launches nothing: the device state is initialised by the first device
+ * call.  Errors: PA_ERR_INVALID_ARG (shape, dtype, alignment, workspace too
+ * small, free_order not a permutation). */
+pa_status pa_pool_create(const pa_pool_desc *desc, pa_pool **out);
+
+/* Release the host state.  Does not touch device buffers (caller-owned);
+ * the caller must make sure no work that uses the pool is still queued. */
+void pa_pool_destroy(pa_pool *pool);
+
+/* Reserve slots so sequence `seq` holds `new_len` tokens, creating it if
+ * it does not exist.  Blocks are taken from the head of the free list only
+ * when the sequence crosses a block boundary ([KVC] paging paragraph; [MKV]
+ * Answer Key item 2).  If the sequence's partly filled tail block is shared
+ * with other sequences and the reservation grows the sequence, the tail is
+ * first copied to a fresh block (copy-on-write, [MKV] Block Tables and
+ * Sharing; [PAS] The bonus: sharing via copy-on-write); the copy covers the
+ * whole block for every layer, K and V, and is enqueued on `stream`.
+ * The number of blocks needed is checked before any change.
+ * Errors: PA_ERR_INVALID_ARG (seq out of range, new_len below the current
+ * length or beyond max_blocks_per_seq * block_size), PA_ERR_NO_BLOCKS,
+ * PA_ERR_CUDA. */
+pa_status pa_alloc_blocks(pa_pool *pool, int32_t seq, int32_t new_len, void *stream);
+
+/* pa_alloc_blocks for n sequences in order, with all copy-on-write copies
+ * of the call in one launch.  Stops at the first failure: sequences before
+ * it are reserved, the failing one and those after it are untouched;
+ * *n_done (always written, even on failure) counts the reserved ones. */
+pa_status pa_alloc_blocks_n(pa_pool *pool, int32_t n, const int32_t *seqs,
+                            const int32_t *new_lens, void *stream, int32_t *n_done);
+
+/* Make `child` share every block of `parent` (reference count + 1 on each);
+ * no data moves ([MKV] Block Tables and Sharing; [PAS] parallel sampling).
+ * Errors: PA_ERR_INVALID_ARG, PA_ERR_NO_SEQ (parent), PA_ERR_SEQ_EXISTS. */
+pa_status pa_fork_cow(pa_pool *pool, int32_t parent, int32_t child);
+
+/* Write one K row and one V row per token into its cache slot of `layer`:
+ *   cache[layer][table[seq][pos / B]][h][pos % B][:] = new[t][h][:]
+ * for t < T and every KV head h.  For an FP8 pool the stored code is
+ * E4M3(round-to-nearest-even, saturate to +-448)(fp32(x) * inv_scale[layer][h])
+ * with the product an IEEE fp32 multiply.  seqs/positions are host arrays of
+ * length T; k_new/v_new are device [T][H_kv][head_dim] act_dtype.  Every
+ * position must lie below the sequence's reserved length and in a block no
+ * other sequence shares (copy-on-write happens in pa_alloc_blocks); (seq,
+ * pos) pairs within one call must be distinct.
+ * Errors: PA_ERR_INVALID_ARG, PA_ERR_NO_SEQ, PA_ERR_SHARED_BLOCK, PA_ERR_CUDA. */
+pa_status pa_append_kv(pa_pool *pool, int32_t layer, int32_t T, const int32_t *seqs,
+                       const int32_t *positions, const void *k_new, const void *v_new,
+                       void *stream);
+
+/* Single-query decode attention through the block tables ([PAS]
+ * PagedAttention: a fused kernel computes attention directly over the
+ * non-contiguous blocks using the block table for addressing):
+ *   out[i][qh][:] = sum_t softmax_t(scale * q[i][qh] . k_t) v_t
+ * over the tokens t < len(seqs[i]) of layer `layer`, with k_t, v_t read from
+ * KV head qh / G (G = num_q_heads / num_kv_heads, 1, 2, 4 or 8), slot t % B of
+ * block table[seqs[i]][t / B].  FP8 values are dequantised as code value x
+ * k_scale / v_scale of (layer, head).  Accumulation is fp32; out is rounded
+ * to act_dtype (nearest even).  seqs is a host array of n sequence ids, each
+ * with length >= 1; q/out are device [n][num_q_heads][head_dim].
+ * partition_tokens: 0 lets the library split long sequences across thread
+ * blocks to balance the GPU (results merged by a log-sum-exp reduction);
+ * -1 never splits; a positive multiple of block_size, at least the pool's
+ * min_partition_tokens, splits every sequence into fixed partitions of that
+ * many tokens.
+ * Errors: PA_ERR_INVALID_ARG, PA_ERR_NO_SEQ, PA_ERR_CUDA. */
+pa_status pa_decode_attention(pa_pool *pool, int32_t layer, int32_t n, const int32_t *seqs,
+                              int32_t num_q_heads, const void *q, void *out, float scale,
+                              int32_t partition_tokens, void *stream);
+
+/* Drop `seq`: every block's reference count falls by one, and blocks that
+ * reach zero go to the tail of the free list in logical-block order ([MKV]
+ * Block Tables and Sharing).  Errors: PA_ERR_INVALID_ARG, PA_ERR_NO_SEQ. */
+pa_status pa_free(pa_pool *pool, int32_t seq);
+
+/* ---- introspection (host state; for tests and schedulers) ---- */
+
+/* Length and block table of `seq`; `table` receives min(cap, nblocks)
+ * entries (may be NULL when cap == 0). */
+pa_status pa_get_seq(pa_pool *pool, int32_t seq, int32_t *len, int32_t *table, int32_t cap,
+                     int32_t *nblocks);
+/* Reference count of every block: `out` holds num_blocks entries. */
+pa_status pa_get_refcounts(pa_pool *pool, int32_t *out, int32_t cap);
+/* Free list from head to tail: `out` receives min(cap, *n) entries. */
+pa_status pa_get_free_list(pa_pool *pool, int32_t *out, int32_t cap, int32_t *n);
+/* Every copy-on-write made so far as (src, dst) pairs: `pairs` receives
+ * min(cap, *n) pairs (2 ints each). */
+pa_status pa_get_cow_log(pa_pool *pool, int32_t *pairs, int32_t cap, int32_t *n);
+/* Number of kernels this pool has launched since it was created. */
+uint64_t pa_launch_count(const pa_pool *pool);
+
+/* Synchronise `stream`, read the device error word, clear it, and store the
+ * PA_DEVERR_* bits in *bits.  Returns PA_ERR_DEVICE_CHECK if any bit was set,
+ * PA_ERR_CUDA if a CUDA call failed, PA_ERR_INVALID_ARG for a host-only pool. */
+pa_status pa_check_device_errors(pa_pool *pool, void *stream, uint32_t *bits);
+
+/* Host-side fault injection for tests: after `n` more block allocations
+ * succeed, further reservations that need blocks fail with PA_ERR_NO_BLOCKS
+ * (state unchanged).  n < 0 switches the fault off. */
+pa_status pa_debug_fail_after(pa_pool *pool, int32_t n);
+
+/* Text of the last failure on the calling thread ("" if none). */
+const char *pa_last_error(void);
+/* Name of a status code. */
+const char *pa_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

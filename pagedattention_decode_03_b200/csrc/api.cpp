@@ -1,0 +1,573 @@
+// C ABI of the paged decode-attention library (declared in include/pa.h).
+//
+// Host side of every call: argument validation, the block manager, planning
+// of the decode work split, and the launches.  Nothing here computes on the
+// CPU what a kernel computes on the GPU; a pool without device buffers
+// (host-only) supports only the block-manager calls.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <optional>
+#include <cstring>
+#include <memory>
+#include <string>
+#include <vector>
+
+#include "block_manager.h"
+#include "pa.h"
+#include "pa_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+pa_status fail(pa_status st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+pa_status cuda_fail(cudaError_t e, const char* what) {
+  g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+  return PA_ERR_CUDA;
+}
+
+constexpr size_t kHeaderBytes = 256;
+constexpr size_t kAlign = 256;
+constexpr int kMinBlocksPerWorker = 4;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int64_t meta_ints(const pa_pool_desc& d) {
+  return static_cast<int64_t>(d.max_seqs) * d.max_blocks_per_seq + d.max_seqs;
+}
+
+int32_t min_partition(const pa_pool_desc& d) {
+  return d.min_partition_tokens > 0 ? d.min_partition_tokens : 512;
+}
+
+int64_t partial_slots(const pa_pool_desc& d) {
+  const int64_t max_tokens = static_cast<int64_t>(d.max_blocks_per_seq) * d.block_size;
+  const int64_t parts = (max_tokens + min_partition(d) - 1) / min_partition(d);
+  const int64_t fixed = static_cast<int64_t>(d.max_seqs) * d.num_kv_heads * parts;
+  return std::max<int64_t>(2 * pa::kMaxWorkers, fixed);
+}
+
+// Switches to the pool's device for the duration of a call.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) {
+      ok = false;
+      return;
+    }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+}  // namespace
+
+struct pa_pool {
+  pa_pool_desc d{};
+  std::unique_ptr<pa::BlockManager> bm;
+  std::vector<pa::CowPair> cow_log;
+  pa::PoolView view{};
+  bool host_only = false;
+  bool dev_ready = false;
+  int num_sms = 0;
+  CUtensorMap tmk{}, tmv{};
+  uint64_t launches = 0;
+  // scratch reused across calls
+  std::vector<pa::CowPair> cows;
+  std::vector<int64_t> slots;
+  std::vector<int32_t> a, b;
+};
+
+namespace {
+
+pa_status ensure_device(pa_pool* p, cudaStream_t stream) {
+  if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
+  if (p->dev_ready) return PA_OK;
+  cudaError_t e = cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, p->d.device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  e = cudaMemsetAsync(p->view.err, 0, sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(error word)");
+
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
+  auto encode = reinterpret_cast<EncodeTiledFn>(fn);
+  const bool fp8 = p->d.kv_dtype == PA_FP8_E4M3;
+  const cuuint64_t rows = static_cast<cuuint64_t>(p->d.num_layers) * p->d.num_blocks *
+                          p->d.num_kv_heads * p->d.block_size;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pa::kHeadDim), rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pa::kHeadDim) * (fp8 ? 1 : 2)};
+  // 128-byte rows of the box: 64 x 16-bit or 128 x 8-bit elements, 16 token rows
+  const cuuint32_t box[2] = {fp8 ? 128u : 64u, 16u};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+  CUresult r = encode(&p->tmk, dt, 2, p->d.k_cache, dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled(k_cache) failed");
+  r = encode(&p->tmv, dt, 2, p->d.v_cache, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled(v_cache) failed");
+  p->dev_ready = true;
+  return PA_OK;
+}
+
+// Ship all pending mirror deltas in a launch of their own.
+pa_status flush_deltas(pa_pool* p, cudaStream_t stream) {
+  pa::MirrorDeltas& md = p->bm->deltas();
+  if (md.size() == 0) return PA_OK;
+  const int n = static_cast<int>(md.size());
+  cudaError_t e = pa::launch_meta_apply(p->view, md.indices().data(), md.values().data(), n, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "meta apply launch");
+  p->launches += (n + pa::kPayloadLarge / 2 - 1) / (pa::kPayloadLarge / 2);
+  md.consume(n);
+  return PA_OK;
+}
+
+pa_status launch_cows(pa_pool* p, cudaStream_t stream) {
+  if (p->cows.empty()) return PA_OK;
+  p->cow_log.insert(p->cow_log.end(), p->cows.begin(), p->cows.end());
+  if (p->host_only) {
+    p->cows.clear();
+    return PA_OK;
+  }
+  DeviceGuard guard(p->d.device);
+  if (!guard.ok) {
+    p->cows.clear();
+    return fail(PA_ERR_CUDA, "cannot select the pool's device");
+  }
+  pa_status st = ensure_device(p, stream);
+  if (st != PA_OK) {
+    p->cows.clear();
+    return st;
+  }
+  pa::MirrorDeltas& md = p->bm->deltas();
+  size_t at = 0;
+  while (at < p->cows.size()) {
+    const size_t n = std::min<size_t>(p->cows.size() - at, 1024);
+    p->a.resize(n);
+    p->b.resize(n);
+    for (size_t k = 0; k < n; ++k) {
+      p->a[k] = p->cows[at + k].src;
+      p->b[k] = p->cows[at + k].dst;
+    }
+    const int nd = static_cast<int>(md.size());
+    int launches = 0;
+    cudaError_t e = pa::launch_cow_copy(p->view, p->a.data(), p->b.data(), static_cast<int>(n),
+                                        md.indices().data(), md.values().data(), nd, stream,
+                                        &launches);
+    p->launches += launches;
+    if (e != cudaSuccess) {
+      p->cows.clear();
+      return cuda_fail(e, "copy-on-write launch");
+    }
+    md.consume(nd);
+    at += n;
+  }
+  p->cows.clear();
+  return PA_OK;
+}
+
+pa_status seq_arg(const pa_pool* p, int32_t seq) {
+  if (seq < 0 || seq >= p->d.max_seqs)
+    return fail(PA_ERR_INVALID_ARG, "sequence id " + std::to_string(seq) + " out of range");
+  return PA_OK;
+}
+
+pa_status bm_status(pa::Status s, const char* what) {
+  switch (s) {
+    case pa::kOk: return PA_OK;
+    case pa::kInvalidArg: return fail(PA_ERR_INVALID_ARG, std::string(what) + ": invalid argument");
+    case pa::kNoBlocks: return fail(PA_ERR_NO_BLOCKS, std::string(what) + ": free list too short");
+    case pa::kNoSeq: return fail(PA_ERR_NO_SEQ, std::string(what) + ": no such sequence");
+    case pa::kSeqExists: return fail(PA_ERR_SEQ_EXISTS, std::string(what) + ": sequence exists");
+    case pa::kSharedBlock:
+      return fail(PA_ERR_SHARED_BLOCK, std::string(what) + ": target block is shared");
+    default: return fail(PA_ERR_INVALID_ARG, what);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t pa_workspace_size(const pa_pool_desc* d) {
+  if (!d || d->max_seqs <= 0 || d->max_blocks_per_seq <= 0 || d->num_kv_heads <= 0 ||
+      d->block_size <= 0)
+    return 0;
+  return kHeaderBytes + align_up(static_cast<size_t>(meta_ints(*d)) * 4) +
+         static_cast<size_t>(partial_slots(*d)) * pa::kPartialSlotFloats * 4;
+}
+
+pa_status pa_pool_create(const pa_pool_desc* d, pa_pool** out) {
+  g_last_error.clear();
+  if (!d || !out) return fail(PA_ERR_INVALID_ARG, "null argument");
+  if (d->head_dim != pa::kHeadDim) return fail(PA_ERR_INVALID_ARG, "head_dim must be 128");
+  if (d->block_size != 16 && d->block_size != 32)
+    return fail(PA_ERR_INVALID_ARG, "block_size must be 16 or 32");
+  if (d->num_layers <= 0 || d->num_kv_heads <= 0 || d->num_blocks <= 0 || d->max_seqs <= 0 ||
+      d->max_blocks_per_seq <= 0)
+    return fail(PA_ERR_INVALID_ARG, "sizes must be positive");
+  if (d->kv_dtype < PA_BF16 || d->kv_dtype > PA_FP8_E4M3)
+    return fail(PA_ERR_INVALID_ARG, "bad kv_dtype");
+  if (d->act_dtype != PA_BF16 && d->act_dtype != PA_FP16)
+    return fail(PA_ERR_INVALID_ARG, "act_dtype must be PA_BF16 or PA_FP16");
+  if (d->kv_dtype != PA_FP8_E4M3 && d->kv_dtype != d->act_dtype)
+    return fail(PA_ERR_INVALID_ARG, "16-bit caches must use the activation dtype");
+  const int64_t rows = static_cast<int64_t>(d->num_layers) * d->num_blocks * d->num_kv_heads *
+                       d->block_size;
+  if (rows >= (int64_t{1} << 31))
+    return fail(PA_ERR_INVALID_ARG, "pool too large: layers*blocks*kv_heads*block_size >= 2^31");
+  if (meta_ints(*d) >= (int64_t{1} << 31)) return fail(PA_ERR_INVALID_ARG, "tables too large");
+  const int32_t pmin = min_partition(*d);
+  if (pmin < d->block_size || pmin % d->block_size != 0)
+    return fail(PA_ERR_INVALID_ARG, "min_partition_tokens must be a multiple of block_size");
+  const bool host_only = d->k_cache == nullptr && d->v_cache == nullptr;
+  if (!host_only) {
+    if (!d->k_cache || !d->v_cache) return fail(PA_ERR_INVALID_ARG, "k_cache and v_cache go together");
+    if ((reinterpret_cast<uintptr_t>(d->k_cache) | reinterpret_cast<uintptr_t>(d->v_cache)) & 15)
+      return fail(PA_ERR_INVALID_ARG, "caches must be 16-byte aligned");
+    if (!d->workspace || (reinterpret_cast<uintptr_t>(d->workspace) & (kAlign - 1)))
+      return fail(PA_ERR_INVALID_ARG, "workspace must be non-null and 256-byte aligned");
+    if (d->workspace_bytes < pa_workspace_size(d))
+      return fail(PA_ERR_INVALID_ARG, "workspace smaller than pa_workspace_size()");
+    if (d->kv_dtype == PA_FP8_E4M3 &&
+        (!d->k_scale || !d->v_scale || !d->k_inv_scale || !d->v_inv_scale))
+      return fail(PA_ERR_INVALID_ARG, "FP8 pools need k/v scales and inverse scales");
+  }
+  if (d->free_order) {
+    std::vector<char> seen(d->num_blocks, 0);
+    for (int32_t k = 0; k < d->num_blocks; ++k) {
+      const int32_t b = d->free_order[k];
+      if (b < 0 || b >= d->num_blocks || seen[b])
+        return fail(PA_ERR_INVALID_ARG, "free_order is not a permutation of the block ids");
+      seen[b] = 1;
+    }
+  }
+  auto p = std::make_unique<pa_pool>();
+  p->d = *d;
+  p->d.min_partition_tokens = pmin;
+  p->d.free_order = nullptr;
+  p->host_only = host_only;
+  p->bm = std::make_unique<pa::BlockManager>(d->num_blocks, d->block_size, d->max_seqs,
+                                             d->max_blocks_per_seq, d->free_order);
+  pa::PoolView& v = p->view;
+  v.k_cache = d->k_cache;
+  v.v_cache = d->v_cache;
+  v.k_scale = d->k_scale;
+  v.v_scale = d->v_scale;
+  v.k_inv = d->k_inv_scale;
+  v.v_inv = d->v_inv_scale;
+  if (!host_only) {
+    uint8_t* ws = static_cast<uint8_t*>(d->workspace);
+    v.err = reinterpret_cast<uint32_t*>(ws);
+    v.meta = reinterpret_cast<int32_t*>(ws + kHeaderBytes);
+    v.tables = v.meta;
+    v.lens = v.meta + static_cast<int64_t>(d->max_seqs) * d->max_blocks_per_seq;
+    v.partials = reinterpret_cast<float*>(ws + kHeaderBytes + align_up(meta_ints(*d) * 4));
+    v.partial_slots = partial_slots(*d);
+  }
+  v.num_layers = d->num_layers;
+  v.num_kv_heads = d->num_kv_heads;
+  v.block_size = d->block_size;
+  v.num_blocks = d->num_blocks;
+  v.max_seqs = d->max_seqs;
+  v.mbps = d->max_blocks_per_seq;
+  v.kv_dtype = d->kv_dtype;
+  v.act_dtype = d->act_dtype;
+  *out = p.release();
+  return PA_OK;
+}
+
+void pa_pool_destroy(pa_pool* p) { delete p; }
+
+pa_status pa_alloc_blocks_n(pa_pool* p, int32_t n, const int32_t* seqs, const int32_t* new_lens,
+                            void* stream, int32_t* n_done) {
+  g_last_error.clear();
+  if (n_done) *n_done = 0;
+  if (!p || n < 0 || (n > 0 && (!seqs || !new_lens)))
+    return fail(PA_ERR_INVALID_ARG, "null argument");
+  p->cows.clear();
+  pa_status st = PA_OK;
+  int32_t k = 0;
+  for (; k < n; ++k) {
+    st = bm_status(p->bm->reserve(seqs[k], new_lens[k], &p->cows), "pa_alloc_blocks");
+    if (st != PA_OK) break;
+  }
+  if (n_done) *n_done = k;
+  const pa_status launch = launch_cows(p, static_cast<cudaStream_t>(stream));
+  return st != PA_OK ? st : launch;
+}
+
+pa_status pa_alloc_blocks(pa_pool* p, int32_t seq, int32_t new_len, void* stream) {
+  int32_t done = 0;
+  return pa_alloc_blocks_n(p, 1, &seq, &new_len, stream, &done);
+}
+
+pa_status pa_fork_cow(pa_pool* p, int32_t parent, int32_t child) {
+  g_last_error.clear();
+  if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
+  return bm_status(p->bm->fork(parent, child), "pa_fork_cow");
+}
+
+pa_status pa_free(pa_pool* p, int32_t seq) {
+  g_last_error.clear();
+  if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
+  return bm_status(p->bm->release(seq), "pa_free");
+}
+
+pa_status pa_append_kv(pa_pool* p, int32_t layer, int32_t T, const int32_t* seqs,
+                       const int32_t* positions, const void* k_new, const void* v_new,
+                       void* stream) {
+  g_last_error.clear();
+  if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
+  if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
+  if (layer < 0 || layer >= p->d.num_layers) return fail(PA_ERR_INVALID_ARG, "layer out of range");
+  if (T < 0 || (T > 0 && (!seqs || !positions || !k_new || !v_new)))
+    return fail(PA_ERR_INVALID_ARG, "null argument");
+  if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & 15)
+    return fail(PA_ERR_INVALID_ARG, "k_new / v_new must be 16-byte aligned");
+  if (T == 0) return PA_OK;
+  p->slots.resize(T);
+  for (int32_t t = 0; t < T; ++t) {
+    pa_status st = seq_arg(p, seqs[t]);
+    if (st != PA_OK) return st;
+    st = bm_status(p->bm->slot(seqs[t], positions[t], &p->slots[t]), "pa_append_kv");
+    if (st != PA_OK) return st;
+  }
+  DeviceGuard guard(p->d.device);
+  if (!guard.ok) return fail(PA_ERR_CUDA, "cannot select the pool's device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  pa_status st = ensure_device(p, s);
+  if (st != PA_OK) return st;
+  pa::MirrorDeltas& md = p->bm->deltas();
+  const int nd = static_cast<int>(md.size());
+  int launches = 0;
+  cudaError_t e = pa::launch_append(p->view, layer, p->slots.data(), T, k_new, v_new,
+                                    md.indices().data(), md.values().data(), nd, s, &launches);
+  p->launches += launches;
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  md.consume(nd);
+  return PA_OK;
+}
+
+pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
+                              int32_t num_q_heads, const void* q, void* out, float scale,
+                              int32_t partition_tokens, void* stream) {
+  g_last_error.clear();
+  if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
+  if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
+  if (layer < 0 || layer >= p->d.num_layers) return fail(PA_ERR_INVALID_ARG, "layer out of range");
+  if (n < 0 || (n > 0 && (!seqs || !q || !out))) return fail(PA_ERR_INVALID_ARG, "null argument");
+  if (p->d.block_size != 16)
+    return fail(PA_ERR_INVALID_ARG, "decode attention supports block_size 16");
+  if (num_q_heads <= 0 || num_q_heads % p->d.num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "num_q_heads must be a multiple of num_kv_heads");
+  const int32_t group = num_q_heads / p->d.num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8)
+    return fail(PA_ERR_INVALID_ARG, "query group (num_q_heads / num_kv_heads) must be 1, 2, 4 or 8");
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 15)
+    return fail(PA_ERR_INVALID_ARG, "q / out must be 16-byte aligned");
+  int mode = pa::kSplitStreamK;
+  int part_blocks = 0;
+  if (partition_tokens == -1) {
+    mode = pa::kSplitNever;
+  } else if (partition_tokens > 0) {
+    if (partition_tokens % p->d.block_size != 0 || partition_tokens < p->d.min_partition_tokens)
+      return fail(PA_ERR_INVALID_ARG,
+                  "partition_tokens must be a multiple of block_size and >= min_partition_tokens");
+    mode = pa::kSplitFixed;
+    part_blocks = partition_tokens / p->d.block_size;
+  } else if (partition_tokens != 0) {
+    return fail(PA_ERR_INVALID_ARG, "partition_tokens must be 0, -1 or positive");
+  }
+  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale must be finite");
+  for (int32_t i = 0; i < n; ++i) {
+    pa_status st = seq_arg(p, seqs[i]);
+    if (st != PA_OK) return st;
+    if (!p->bm->active(seqs[i])) return fail(PA_ERR_NO_SEQ, "pa_decode_attention: no such sequence");
+    if (p->bm->len(seqs[i]) < 1) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: empty sequence");
+  }
+  if (n == 0) return PA_OK;
+  DeviceGuard guard(p->d.device);
+  if (!guard.ok) return fail(PA_ERR_CUDA, "cannot select the pool's device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  pa_status st = ensure_device(p, s);
+  if (st != PA_OK) return st;
+  st = flush_deltas(p, s);
+  if (st != PA_OK) return st;
+
+  const int H = p->d.num_kv_heads;
+  const int cap = pa::decode_worker_capacity(p->d.kv_dtype, group, p->num_sms);
+  const int64_t slots_cap = p->view.partial_slots;
+  pa::DecodeArgs args;
+  args.q = q;
+  args.out = out;
+  args.layer = layer;
+  args.num_q_heads = num_q_heads;
+  args.group = group;
+  args.scale = scale;
+  args.q_item_stride = static_cast<int64_t>(num_q_heads) * pa::kHeadDim;
+  static thread_local pa::DecodePlan plan;
+  int32_t at = 0;
+  while (at < n) {
+    // Items of this launch: up to the parameter capacity, and (fixed mode) the
+    // partial slots the workspace holds.
+    int32_t cnt = 0;
+    int64_t work = 0;
+    plan.pre[0] = 0;
+    while (at + cnt < n && cnt < pa::kDecodeItemsCap) {
+      const int32_t len = p->bm->len(seqs[at + cnt]);
+      const int32_t nb = (len + 15) / 16;
+      int64_t units = nb;
+      if (mode == pa::kSplitFixed) units = (nb + part_blocks - 1) / part_blocks;
+      if (mode == pa::kSplitNever) units = 1;
+      if (mode == pa::kSplitFixed && cnt > 0 && (work + units) * H > slots_cap) break;
+      if (mode == pa::kSplitFixed && units * H > slots_cap)
+        return fail(PA_ERR_INVALID_ARG, "partition_tokens too small for the workspace");
+      plan.seq[cnt] = seqs[at + cnt];
+      work += units;
+      plan.pre[cnt + 1] = static_cast<int32_t>(work);
+      ++cnt;
+    }
+    plan.n = cnt;
+    plan.mode = mode;
+    plan.part_blocks = part_blocks;
+    plan.per_head = work;
+    const int64_t total = work * H;
+    int64_t W = std::min<int64_t>(cap, total);
+    if (mode == pa::kSplitStreamK) {
+      W = std::min<int64_t>(W, std::max<int64_t>(1, (total + kMinBlocksPerWorker - 1) / kMinBlocksPerWorker));
+      W = std::min<int64_t>(W, slots_cap / 2);
+    }
+    plan.workers = static_cast<int32_t>(std::max<int64_t>(1, W));
+    args.item_offset = at;
+    int launches = 0;
+    cudaError_t e = pa::launch_decode(p->view, &p->tmk, &p->tmv, plan, args, s, &launches);
+    p->launches += launches;
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    at += cnt;
+  }
+  return PA_OK;
+}
+
+pa_status pa_get_seq(pa_pool* p, int32_t seq, int32_t* len, int32_t* table, int32_t cap,
+                     int32_t* nblocks) {
+  g_last_error.clear();
+  if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
+  pa_status st = seq_arg(p, seq);
+  if (st != PA_OK) return st;
+  if (!p->bm->active(seq)) return fail(PA_ERR_NO_SEQ, "pa_get_seq: no such sequence");
+  const std::vector<int32_t>& t = p->bm->table(seq);
+  if (cap > 0 && !table) return fail(PA_ERR_INVALID_ARG, "null table with cap > 0");
+  const int32_t m = std::min<int32_t>(cap, static_cast<int32_t>(t.size()));
+  if (m > 0) std::memcpy(table, t.data(), sizeof(int32_t) * m);
+  if (len) *len = p->bm->len(seq);
+  if (nblocks) *nblocks = static_cast<int32_t>(t.size());
+  return PA_OK;
+}
+
+pa_status pa_get_refcounts(pa_pool* p, int32_t* out, int32_t cap) {
+  g_last_error.clear();
+  if (!p || !out) return fail(PA_ERR_INVALID_ARG, "null argument");
+  if (cap < p->d.num_blocks) return fail(PA_ERR_INVALID_ARG, "cap < num_blocks");
+  for (int32_t b = 0; b < p->d.num_blocks; ++b) out[b] = p->bm->refcount(b);
+  return PA_OK;
+}
+
+pa_status pa_get_free_list(pa_pool* p, int32_t* out, int32_t cap, int32_t* n) {
+  g_last_error.clear();
+  if (!p || !n || (cap > 0 && !out)) return fail(PA_ERR_INVALID_ARG, "null argument");
+  std::vector<int32_t> fl;
+  p->bm->free_list(&fl);
+  const int32_t m = std::min<int32_t>(cap, static_cast<int32_t>(fl.size()));
+  if (m > 0) std::memcpy(out, fl.data(), sizeof(int32_t) * m);
+  *n = static_cast<int32_t>(fl.size());
+  return PA_OK;
+}
+
+pa_status pa_get_cow_log(pa_pool* p, int32_t* pairs, int32_t cap, int32_t* n) {
+  g_last_error.clear();
+  if (!p || !n || (cap > 0 && !pairs)) return fail(PA_ERR_INVALID_ARG, "null argument");
+  const int32_t m = std::min<int32_t>(cap, static_cast<int32_t>(p->cow_log.size()));
+  for (int32_t k = 0; k < m; ++k) {
+    pairs[2 * k] = p->cow_log[k].src;
+    pairs[2 * k + 1] = p->cow_log[k].dst;
+  }
+  *n = static_cast<int32_t>(p->cow_log.size());
+  return PA_OK;
+}
+
+uint64_t pa_launch_count(const pa_pool* p) { return p ? p->launches : 0; }
+
+pa_status pa_check_device_errors(pa_pool* p, void* stream, uint32_t* bits) {
+  g_last_error.clear();
+  if (!p || !bits) return fail(PA_ERR_INVALID_ARG, "null argument");
+  if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
+  DeviceGuard guard(p->d.device);
+  if (!guard.ok) return fail(PA_ERR_CUDA, "cannot select the pool's device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!p->dev_ready) {
+    *bits = 0;
+    return PA_OK;
+  }
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  uint32_t v = 0;
+  e = cudaMemcpy(&v, p->view.err, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  e = cudaMemset(p->view.err, 0, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+  *bits = v;
+  if (v) {
+    char buf[96];
+    std::snprintf(buf, sizeof(buf), "device check failed: bits 0x%x", v);
+    return fail(PA_ERR_DEVICE_CHECK, buf);
+  }
+  return PA_OK;
+}
+
+pa_status pa_debug_fail_after(pa_pool* p, int32_t n) {
+  g_last_error.clear();
+  if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
+  p->bm->set_fail_after(n);
+  return PA_OK;
+}
+
+const char* pa_last_error(void) { return g_last_error.c_str(); }
+
+const char* pa_status_string(int32_t s) {
+  switch (s) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+    case PA_ERR_NO_BLOCKS: return "PA_ERR_NO_BLOCKS";
+    case PA_ERR_NO_SEQ: return "PA_ERR_NO_SEQ";
+    case PA_ERR_SEQ_EXISTS: return "PA_ERR_SEQ_EXISTS";
+    case PA_ERR_SHARED_BLOCK: return "PA_ERR_SHARED_BLOCK";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    case PA_ERR_DEVICE_CHECK: return "PA_ERR_DEVICE_CHECK";
+    default: return "PA_UNKNOWN_STATUS";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,919 @@
+// Paged single-query decode attention for sm_100a.
+//
+// Computes, for every (sequence, query head),
+//     out = sum_t softmax_t(scale * q . k_t) v_t      over t < len(seq),
+// reading k_t, v_t from slot t % B of physical block table[seq][t / B] of the
+// query head's KV head -- attention taken directly over the non-contiguous
+// blocks, addressed through the block table (kv-cache-pagedattention-serving,
+// PagedAttention: virtual memory for GPUs; "Managing the KV Cache", Block
+// Tables and Sharing: the kernel gathers K/V through the block table).
+//
+// Design (B200-first; the pages give no kernel design):
+//   * Work unit = (sequence, KV head); the G = H_q / H_kv query heads of the
+//     group are processed together, so every K/V byte is read once.
+//   * Each warp is an independent worker with its own ring of shared-memory
+//     stages.  One (layer, block, head) K tile and its V tile are one stage,
+//     fetched by TMA tensor loads (cp.async.bulk.tensor, 128-byte swizzle)
+//     that complete on a per-stage mbarrier; the warp keeps STAGES tiles in
+//     flight while it computes on the oldest.  Block ids come from the device
+//     mirror of the block tables, cached 32 at a time in registers.
+//   * G >= 4: QK^T and P.V are warp-level tensor-core MMAs (m16n8k16) with the
+//     16 tokens of a block on M and the (padded) query group on N; S^T stays in
+//     registers, the online softmax runs on the accumulator fragments, and P^T
+//     reaches the PV MMA through movmatrix.  G <= 2: fp32 FMAs on CUDA cores.
+//   * Work is spread over all warps of the GPU in equal shares of KV blocks
+//     (stream-K style): a worker's share can start and end inside a sequence;
+//     partial results (running max m, sum l, unnormalised o) are merged by a
+//     small log-sum-exp reduction kernel.  Fixed-size partitions and "never
+//     split" are the two other modes.
+//   * FP8 E4M3 KV: tiles are half the bytes; codes are converted to f16 with
+//     the hardware cvt (exact), K's scale is folded into the logit scale and
+//     V's into the output.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <type_traits>
+
+#include "device_common.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+constexpr int kWarps = 4;              // warps (independent workers) per CTA
+constexpr int kBlock = 16;             // tokens per KV block handled by the kernel
+constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int KV>
+struct Tile {
+  static constexpr int kBytes = KV == kFP8 ? kBlock * kHeadDim : kBlock * kHeadDim * 2;  // one K or V tile
+  static constexpr int kStageBytes = 2 * kBytes;
+  static constexpr int kStages = KV == kFP8 ? 6 : 3;
+  static constexpr int kRingBytes = kStages * kStageBytes;
+};
+
+struct DecodeKParams {
+  const uint8_t* q;
+  uint8_t* out;
+  const int32_t* tables;
+  const int32_t* lens;
+  float* partials;
+  uint32_t* err;
+  const float* k_scale;
+  const float* v_scale;
+  int64_t q_item_stride;   // elements between items of q / out
+  float scale;
+  int32_t layer, num_kv_heads, num_blocks, mbps, group;
+  int64_t total;           // work units over all heads
+  DecodePlan plan;
+};
+
+struct Seg {
+  int32_t h, i, b0, b1, dest, len, seq;
+  bool valid;
+};
+
+// Index of the item whose prefix range holds r: pre[i] <= r < pre[i+1].
+__device__ __forceinline__ int find_item(const DecodePlan& P, int64_t r) {
+  int lo = 0, hi = P.n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (P.pre[mid] <= r) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int64_t worker_start(int64_t total, int w, int W) {
+  return (total * w) / W;
+}
+
+// Next segment of a worker whose remaining range is [g, g_end).
+__device__ __forceinline__ Seg next_seg(const DecodeKParams& prm, int64_t& g, int64_t g_end,
+                                        int w, bool first) {
+  Seg s;
+  s.valid = g < g_end;
+  if (!s.valid) return s;
+  const DecodePlan& P = prm.plan;
+  const int64_t per_head = P.per_head;
+  s.h = static_cast<int32_t>(g / per_head);
+  const int64_t r = g - static_cast<int64_t>(s.h) * per_head;
+  if (P.mode == kSplitNever) {
+    s.i = static_cast<int32_t>(r);
+  } else {
+    s.i = find_item(P, r);
+  }
+  s.seq = P.seq[s.i];
+  s.len = prm.lens[s.seq];
+  int32_t nb = (s.len + kBlock - 1) / kBlock;
+  if (s.len <= 0 || nb > prm.mbps) {
+    atomicOr(prm.err, kErrBadLen);
+    nb = min(max(nb, 1), prm.mbps);
+    s.len = max(s.len, 1);
+  }
+  if (P.mode == kSplitStreamK) {
+    const int32_t unit_nb = P.pre[s.i + 1] - P.pre[s.i];
+    if (unit_nb != nb) atomicOr(prm.err, kErrBadLen);
+    s.b0 = static_cast<int32_t>(r - P.pre[s.i]);
+    const int64_t take = min(static_cast<int64_t>(unit_nb - s.b0), g_end - g);
+    s.b1 = s.b0 + static_cast<int32_t>(take);
+    const bool whole = s.b0 == 0 && s.b1 == unit_nb;
+    s.dest = whole ? -1 : (first ? 2 * w : 2 * w + 1);
+    g += take;
+  } else if (P.mode == kSplitFixed) {
+    const int32_t p = static_cast<int32_t>(r - P.pre[s.i]);
+    const int32_t np = P.pre[s.i + 1] - P.pre[s.i];
+    s.b0 = p * P.part_blocks;
+    s.b1 = min(nb, s.b0 + P.part_blocks);
+    if (s.b0 >= s.b1) {  // inconsistent lengths: clamp to an empty-free range
+      atomicOr(prm.err, kErrBadLen);
+      s.b0 = max(0, s.b1 - 1);
+    }
+    s.dest = np == 1 ? -1 : static_cast<int32_t>(g);
+    g += 1;
+  } else {
+    s.b0 = 0;
+    s.b1 = nb;
+    s.dest = -1;
+    g += 1;
+  }
+  return s;
+}
+
+// ------------------------------------------------------------------ producer
+template <int KV>
+struct Producer {
+  int64_t g, g_end;
+  Seg seg;
+  int32_t b;          // next block of seg to fetch
+  bool first;
+  int32_t tc_val, tc_base, tc_seq;
+  uint32_t issued;
+
+  __device__ __forceinline__ void init(const DecodeKParams& prm, int64_t g0, int64_t g1, int w) {
+    g = g0;
+    g_end = g1;
+    first = true;
+    seg = next_seg(prm, g, g_end, w, first);
+    first = false;
+    b = seg.b0;
+    tc_seq = -1;
+    tc_base = 0;
+    tc_val = 0;
+    issued = 0;
+  }
+
+  // Fetch the next block of this worker into stage issued % kStages.
+  __device__ __forceinline__ void issue(const DecodeKParams& prm, const CUtensorMap* tmk,
+                                        const CUtensorMap* tmv, uint32_t ring, uint32_t bars,
+                                        int w, int lane) {
+    if (!seg.valid) return;
+    if (b == seg.b1) {
+      seg = next_seg(prm, g, g_end, w, false);
+      if (!seg.valid) return;
+      b = seg.b0;
+    }
+    if (seg.seq != tc_seq || b < tc_base || b >= tc_base + 32) {
+      tc_seq = seg.seq;
+      tc_base = b;
+      const int idx = b + lane;
+      tc_val = idx < prm.mbps ? prm.tables[static_cast<int64_t>(seg.seq) * prm.mbps + idx] : 0;
+    }
+    int32_t phys = __shfl_sync(0xffffffffu, tc_val, b - tc_base);
+    if (static_cast<uint32_t>(phys) >= static_cast<uint32_t>(prm.num_blocks)) {
+      if (lane == 0) atomicOr(prm.err, kErrBadBlock);
+      phys = 0;
+    }
+    const uint32_t stage = issued % Tile<KV>::kStages;
+    const uint32_t bar = bars + stage * 8;
+    const uint32_t dst = ring + stage * Tile<KV>::kStageBytes;
+    const int32_t row =
+        ((prm.layer * prm.num_blocks + phys) * prm.num_kv_heads + seg.h) * kBlock;
+    if (lane == 0) {
+      dev::mbar_arrive_expect_tx(bar, Tile<KV>::kStageBytes);
+      if constexpr (KV == kFP8) {
+        dev::tma_load_2d(dst, tmk, 0, row, bar);
+        dev::tma_load_2d(dst + Tile<KV>::kBytes, tmv, 0, row, bar);
+      } else {
+        dev::tma_load_2d(dst, tmk, 0, row, bar);
+        dev::tma_load_2d(dst + 2048, tmk, 64, row, bar);
+        dev::tma_load_2d(dst + Tile<KV>::kBytes, tmv, 0, row, bar);
+        dev::tma_load_2d(dst + Tile<KV>::kBytes + 2048, tmv, 64, row, bar);
+      }
+    }
+    ++issued;
+    ++b;
+  }
+};
+
+// Zero V rows [nvalid, 16) of a staged tile so masked tokens contribute exact
+// zeros whatever stale bits the slots hold.
+template <int KV>
+__device__ __forceinline__ void zero_tail_rows(uint8_t* vtile, int nvalid, int lane) {
+  constexpr int kRowChunks = KV == kFP8 ? 8 : 16;  // 16-byte chunks per token row
+  const int n = (kBlock - nvalid) * kRowChunks;
+  for (int c = lane; c < n; c += 32) {
+    const int t = nvalid + c / kRowChunks;
+    const int k = c % kRowChunks;
+    uint8_t* p;
+    if constexpr (KV == kFP8) {
+      p = vtile + t * 128 + k * 16;
+    } else {
+      p = vtile + (k >> 3) * 2048 + t * 128 + (k & 7) * 16;
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(0, 0, 0, 0);
+  }
+  dev::fence_proxy_async_smem();
+  __syncwarp();
+}
+
+__device__ __forceinline__ float warp_max_rows(float x) {  // over lanes sharing lane & 3
+  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
+  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
+  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
+  return x;
+}
+__device__ __forceinline__ float warp_sum_rows(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 4);
+  x += __shfl_xor_sync(0xffffffffu, x, 8);
+  x += __shfl_xor_sync(0xffffffffu, x, 16);
+  return x;
+}
+
+template <int ACT>
+__device__ __forceinline__ float act_to_f32(uint16_t x) {
+  if constexpr (ACT == kBF16) return __uint_as_float(static_cast<uint32_t>(x) << 16);
+  else return __half2float(__ushort_as_half(x));
+}
+
+template <int ACT>
+__device__ __forceinline__ uint16_t f32_to_act(float x) {
+  if constexpr (ACT == kBF16) return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+  else return __half_as_ushort(__float2half_rn(x));
+}
+
+// ============================================================ tensor-core path
+// Query group of G in {4, 8} query heads on the MMA N dimension (8 columns).
+template <int KV, int ACT, int G>
+struct MmaPath {
+  static constexpr bool kF16 = (KV == kFP16) || (KV == kFP8);
+  uint32_t qf[8][2];   // Q^T B-fragments for the 8 k-steps
+  float o[8][4];       // O^T accumulators: 8 m-tiles (d) x (2 heads per lane)
+  float m0, m1, l0, l1;
+  float sl2;           // logit scale in log2 units
+  float vmul;          // V dequantisation scale (1 for 16-bit KV)
+
+  __device__ __forceinline__ void begin(const DecodeKParams& prm, const Seg& s, int lane) {
+    const int g = lane >> 2, tig = lane & 3;
+    const int item = s.i;  // item index within this launch
+    const uint16_t* qrow = reinterpret_cast<const uint16_t*>(prm.q) +
+                           item * prm.q_item_stride + (s.h * G + g) * kHeadDim;
+    float qscale = 1.f;
+    sl2 = prm.scale * kLog2e;
+    vmul = 1.f;
+    if constexpr (KV == kFP8) {
+      // Q is pre-multiplied by the softmax scale before rounding to f16; K's
+      // dequantisation scale is folded into the logit scale.
+      qscale = prm.scale;
+      sl2 = prm.k_scale[prm.layer * prm.num_kv_heads + s.h] * kLog2e;
+      vmul = prm.v_scale[prm.layer * prm.num_kv_heads + s.h];
+    }
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      if (g < G) {
+        if constexpr (KV == kFP8) {
+          const uint2 raw = *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * tig);
+          const float a = act_to_f32<ACT>(raw.x & 0xffff) * qscale;
+          const float b = act_to_f32<ACT>(raw.x >> 16) * qscale;
+          const float c = act_to_f32<ACT>(raw.y & 0xffff) * qscale;
+          const float d = act_to_f32<ACT>(raw.y >> 16) * qscale;
+          qf[ks][0] = dev::pack_f16(a, b);
+          qf[ks][1] = dev::pack_f16(c, d);
+        } else {
+          qf[ks][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tig);
+          qf[ks][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * tig);
+        }
+      } else {
+        qf[ks][0] = 0u;
+        qf[ks][1] = 0u;
+      }
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.f;
+  }
+
+  __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    if constexpr (kF16) dev::mma_f16(d, a, b0, b1);
+    else dev::mma_bf16(d, a, b0, b1);
+  }
+
+  __device__ __forceinline__ void block(uint32_t ks_addr, uint32_t vs_addr, int nvalid, int lane) {
+    const int g = lane >> 2, tig = lane & 3;
+    const int r8 = lane & 7, j = lane >> 3;
+    // ---- S^T = K Q^T : 16 tokens x 8 heads
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      const int tok = r8 + ((j & 1) << 3);
+      const int add = j >> 1;
+      if constexpr (KV == kFP8) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          uint32_t R[4];
+          dev::ldsm_x4(ks_addr + tok * 128 + (((2 * kk + add) ^ r8) << 4), R);
+          uint32_t a0[4] = {dev::e4m3x2_to_f16x2(R[0] & 0xffff), dev::e4m3x2_to_f16x2(R[1] & 0xffff),
+                            dev::e4m3x2_to_f16x2(R[0] >> 16), dev::e4m3x2_to_f16x2(R[1] >> 16)};
+          uint32_t a1[4] = {dev::e4m3x2_to_f16x2(R[2] & 0xffff), dev::e4m3x2_to_f16x2(R[3] & 0xffff),
+                            dev::e4m3x2_to_f16x2(R[2] >> 16), dev::e4m3x2_to_f16x2(R[3] >> 16)};
+          mma(sa, a0, qf[2 * kk][0], qf[2 * kk][1]);
+          mma(sb, a1, qf[2 * kk + 1][0], qf[2 * kk + 1][1]);
+        }
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const int chunk = 2 * ks + add;
+          uint32_t a[4];
+          dev::ldsm_x4(ks_addr + (ks >> 2) * 2048 + tok * 128 + (((chunk & 7) ^ r8) << 4), a);
+          if (ks & 1) mma(sb, a, qf[ks][0], qf[ks][1]);
+          else mma(sa, a, qf[ks][0], qf[ks][1]);
+        }
+      }
+    }
+    float s0 = (sa[0] + sb[0]) * sl2, s1 = (sa[1] + sb[1]) * sl2;  // token g, heads 2tig, 2tig+1
+    float s2 = (sa[2] + sb[2]) * sl2, s3 = (sa[3] + sb[3]) * sl2;  // token g+8
+    if (nvalid < kBlock) {
+      if (g >= nvalid) s0 = s1 = -INFINITY;
+      if (g + 8 >= nvalid) s2 = s3 = -INFINITY;
+    }
+    // ---- online softmax over the 16 tokens (rows) per head (column)
+    const float mx0 = warp_max_rows(fmaxf(s0, s2));
+    const float mx1 = warp_max_rows(fmaxf(s1, s3));
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float c0 = dev::exp2_approx(m0 - mn0), c1 = dev::exp2_approx(m1 - mn1);
+    m0 = mn0;
+    m1 = mn1;
+    const float p0 = dev::exp2_approx(s0 - mn0), p1 = dev::exp2_approx(s1 - mn1);
+    const float p2 = dev::exp2_approx(s2 - mn0), p3 = dev::exp2_approx(s3 - mn1);
+    l0 = l0 * c0 + p0 + p2;
+    l1 = l1 * c1 + p1 + p3;
+    if (__any_sync(0xffffffffu, c0 != 1.f || c1 != 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        o[mt][0] *= c0;
+        o[mt][1] *= c1;
+        o[mt][2] *= c0;
+        o[mt][3] *= c1;
+      }
+    }
+    // ---- P^T as the B operand of O^T += V^T P^T
+    const uint32_t x0 = kF16 ? dev::pack_f16(p0, p1) : dev::pack_bf16(p0, p1);
+    const uint32_t x1 = kF16 ? dev::pack_f16(p2, p3) : dev::pack_bf16(p2, p3);
+    const uint32_t pb0 = dev::movm_t(x0);
+    const uint32_t pb1 = dev::movm_t(x1);
+    if constexpr (KV == kFP8) {
+      const int tok = r8 + ((j & 1) << 3);
+      const int add = j >> 1;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t R[4];
+        dev::ldsm_x4_t(vs_addr + tok * 128 + (((2 * cc + add) ^ r8) << 4), R);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t X0 = dev::prmt(R[2 * half], 0, 0x3120);
+          const uint32_t X1 = dev::prmt(R[2 * half + 1], 0, 0x3120);
+          uint32_t a[4] = {dev::e4m3x2_to_f16x2(X0 & 0xffff), dev::e4m3x2_to_f16x2(X0 >> 16),
+                           dev::e4m3x2_to_f16x2(X1 & 0xffff), dev::e4m3x2_to_f16x2(X1 >> 16)};
+          mma(o[2 * cc + half], a, pb0, pb1);
+        }
+      }
+    } else {
+      const int tok = r8 + ((j >> 1) << 3);
+      const int add = j & 1;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const int chunk = 2 * mt + add;
+        uint32_t a[4];
+        dev::ldsm_x4_t(vs_addr + (mt >> 2) * 2048 + tok * 128 + (((chunk & 7) ^ r8) << 4), a);
+        mma(o[mt], a, pb0, pb1);
+      }
+    }
+  }
+
+  // d index of accumulator o[mt][k] (k = 0,1: first row; 2,3: second row).
+  __device__ __forceinline__ static int d_of(int mt, int second, int g) {
+    if constexpr (KV == kFP8) return 16 * mt + 2 * g + second;
+    else return 16 * mt + 8 * second + g;
+  }
+
+  __device__ __forceinline__ void finish(const DecodeKParams& prm, const Seg& s, int lane) {
+    const int g = lane >> 2, tig = lane & 3;
+    const float lt0 = warp_sum_rows(l0), lt1 = warp_sum_rows(l1);
+    const int h0 = 2 * tig, h1 = 2 * tig + 1;
+    if (s.dest < 0) {
+      uint16_t* orow = reinterpret_cast<uint16_t*>(prm.out) + s.i * prm.q_item_stride +
+                       (s.h * G) * kHeadDim;
+      const float f0 = vmul / lt0, f1 = vmul / lt1;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+#pragma unroll
+        for (int sec = 0; sec < 2; ++sec) {
+          const int d = d_of(mt, sec, g);
+          if (h0 < G) orow[h0 * kHeadDim + d] = f32_to_act<ACT>(o[mt][2 * sec] * f0);
+          if (h1 < G) orow[h1 * kHeadDim + d] = f32_to_act<ACT>(o[mt][2 * sec + 1] * f1);
+        }
+      }
+    } else {
+      float* slot = prm.partials + static_cast<int64_t>(s.dest) * kPartialSlotFloats;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+#pragma unroll
+        for (int sec = 0; sec < 2; ++sec) {
+          const int d = d_of(mt, sec, g);
+          if (h0 < G) slot[h0 * kHeadDim + d] = o[mt][2 * sec] * vmul;
+          if (h1 < G) slot[h1 * kHeadDim + d] = o[mt][2 * sec + 1] * vmul;
+        }
+      }
+      if (g == 0) {
+        float* ml = slot + kMaxGroup * kHeadDim;
+        if (h0 < G) { ml[2 * h0] = m0; ml[2 * h0 + 1] = lt0; }
+        if (h1 < G) { ml[2 * h1] = m1; ml[2 * h1 + 1] = lt1; }
+      }
+    }
+  }
+};
+
+// =============================================================== CUDA-core path
+// G in {1, 2}: lane = (token row r = lane / 4, d-quarter qd = lane % 4); a
+// block is processed as two halves (tokens r and r + 8).
+template <int KV, int ACT, int G>
+struct FmaPath {
+  // 16-bit KV: each lane covers 32 d as 4 chunks of 8; FP8: 2 chunks of 16.
+  static constexpr int kChunks = KV == kFP8 ? 2 : 4;
+  static constexpr int kPer = KV == kFP8 ? 16 : 8;
+  float qv[G][kChunks][kPer];
+  float acc[G][kChunks][kPer];
+  float m[G], l[G];
+  float sl2, vmul;
+
+  // chunk position (16-byte unit within the 128-byte row of its box) and box
+  __device__ __forceinline__ static int cib(int qd, int i) {
+    if constexpr (KV == kFP8) return 2 * qd + i;
+    else return 4 * (qd & 1) + ((i + 2 * (qd >> 1)) & 3);
+  }
+  __device__ __forceinline__ static int d0_of(int qd, int i) {
+    if constexpr (KV == kFP8) return 16 * (2 * qd + i);
+    else return 64 * (qd >> 1) + 8 * cib(qd, i);
+  }
+  __device__ __forceinline__ static uint32_t row_addr(uint32_t base, int t, int qd, int i) {
+    if constexpr (KV == kFP8) return base + t * 128 + ((cib(qd, i) ^ (t & 7)) << 4);
+    else return base + (qd >> 1) * 2048 + t * 128 + ((cib(qd, i) ^ (t & 7)) << 4);
+  }
+
+  __device__ __forceinline__ void to_f32(const uint4& raw, float (&f)[kPer]) {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    if constexpr (KV == kFP8) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t lo = dev::e4m3x2_to_f16x2(w[k] & 0xffff);
+        const uint32_t hi = dev::e4m3x2_to_f16x2(w[k] >> 16);
+        f[4 * k + 0] = dev::f16lo_to_f32(lo);
+        f[4 * k + 1] = dev::f16hi_to_f32(lo);
+        f[4 * k + 2] = dev::f16lo_to_f32(hi);
+        f[4 * k + 3] = dev::f16hi_to_f32(hi);
+      }
+    } else if constexpr (KV == kBF16) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        f[2 * k] = dev::bf16lo_to_f32(w[k]);
+        f[2 * k + 1] = dev::bf16hi_to_f32(w[k]);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        f[2 * k] = dev::f16lo_to_f32(w[k]);
+        f[2 * k + 1] = dev::f16hi_to_f32(w[k]);
+      }
+    }
+  }
+
+  __device__ __forceinline__ void begin(const DecodeKParams& prm, const Seg& s, int lane) {
+    const int qd = lane & 3;
+    sl2 = prm.scale * kLog2e;
+    vmul = 1.f;
+    if constexpr (KV == kFP8) {
+      sl2 *= prm.k_scale[prm.layer * prm.num_kv_heads + s.h];
+      vmul = prm.v_scale[prm.layer * prm.num_kv_heads + s.h];
+    }
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      const uint16_t* qrow = reinterpret_cast<const uint16_t*>(prm.q) + s.i * prm.q_item_stride +
+                             (s.h * G + gg) * kHeadDim;
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const uint16_t* src = qrow + d0_of(qd, i);
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) qv[gg][i][e] = act_to_f32<ACT>(src[e]);
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[gg][i][e] = 0.f;
+      }
+      m[gg] = -INFINITY;
+      l[gg] = 0.f;
+    }
+  }
+
+  __device__ __forceinline__ void block(uint32_t ks_addr, uint32_t vs_addr, int nvalid, int lane) {
+    const int r = lane >> 2, qd = lane & 3;
+    float s[2][G];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int t = r + 8 * half;
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) s[half][gg] = 0.f;
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        uint4 raw;
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w)
+                     : "r"(row_addr(ks_addr, t, qd, i)));
+        float kf[kPer];
+        to_f32(raw, kf);
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg)
+#pragma unroll
+          for (int e = 0; e < kPer; ++e) s[half][gg] = fmaf(qv[gg][i][e], kf[e], s[half][gg]);
+      }
+    }
+#pragma unroll
+    for (int half = 0; half < 2; ++half)
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) {
+        float x = s[half][gg];
+        x += __shfl_xor_sync(0xffffffffu, x, 1);
+        x += __shfl_xor_sync(0xffffffffu, x, 2);
+        x *= sl2;
+        if (r + 8 * half >= nvalid) x = -INFINITY;
+        s[half][gg] = x;
+      }
+    float p[2][G];
+    bool rescale = false;
+    float corr[G];
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      const float mx = warp_max_rows(fmaxf(s[0][gg], s[1][gg]));
+      const float mn = fmaxf(m[gg], mx);
+      corr[gg] = dev::exp2_approx(m[gg] - mn);
+      m[gg] = mn;
+      p[0][gg] = dev::exp2_approx(s[0][gg] - mn);
+      p[1][gg] = dev::exp2_approx(s[1][gg] - mn);
+      l[gg] = l[gg] * corr[gg] + p[0][gg] + p[1][gg];
+      rescale |= corr[gg] != 1.f;
+    }
+    if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg)
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i)
+#pragma unroll
+          for (int e = 0; e < kPer; ++e) acc[gg][i][e] *= corr[gg];
+    }
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int t = r + 8 * half;
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        uint4 raw;
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w)
+                     : "r"(row_addr(vs_addr, t, qd, i)));
+        float vf[kPer];
+        to_f32(raw, vf);
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg)
+#pragma unroll
+          for (int e = 0; e < kPer; ++e) acc[gg][i][e] = fmaf(p[half][gg], vf[e], acc[gg][i][e]);
+      }
+    }
+  }
+
+  __device__ __forceinline__ void finish(const DecodeKParams& prm, const Seg& s, int lane) {
+    const int r = lane >> 2, qd = lane & 3;
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      l[gg] = warp_sum_rows(l[gg]);
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i)
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[gg][i][e] = warp_sum_rows(acc[gg][i][e]);
+    }
+    // lanes with r < kChunks write chunk i = r of their d-quarter
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        if (r != i) continue;
+        const int d0 = d0_of(qd, i);
+        if (s.dest < 0) {
+          uint16_t* orow = reinterpret_cast<uint16_t*>(prm.out) + s.i * prm.q_item_stride +
+                           (s.h * G + gg) * kHeadDim + d0;
+          const float f = vmul / l[gg];
+#pragma unroll
+          for (int e = 0; e < kPer; e += 2) {
+            const uint32_t two = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg][i][e] * f)) |
+                                 (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg][i][e + 1] * f)) << 16);
+            *reinterpret_cast<uint32_t*>(orow + e) = two;
+          }
+        } else {
+          float* slot = prm.partials + static_cast<int64_t>(s.dest) * kPartialSlotFloats +
+                        gg * kHeadDim + d0;
+#pragma unroll
+          for (int e = 0; e < kPer; e += 4)
+            *reinterpret_cast<float4*>(slot + e) =
+                make_float4(acc[gg][i][e] * vmul, acc[gg][i][e + 1] * vmul,
+                            acc[gg][i][e + 2] * vmul, acc[gg][i][e + 3] * vmul);
+        }
+      }
+    }
+    if (s.dest >= 0 && lane == 0) {
+      float* ml = prm.partials + static_cast<int64_t>(s.dest) * kPartialSlotFloats +
+                  kMaxGroup * kHeadDim;
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) {
+        ml[2 * gg] = m[gg];
+        ml[2 * gg + 1] = l[gg];
+      }
+    }
+  }
+};
+
+template <int KV, int ACT, int G>
+using PathFor = typename std::conditional<(G >= 4), MmaPath<KV, ACT, G>, FmaPath<KV, ACT, G>>::type;
+
+// ===================================================================== kernel
+template <int KV, int ACT, int G>
+__global__ void __launch_bounds__(kWarps * 32)
+    decode_kernel(const __grid_constant__ DecodeKParams prm, const __grid_constant__ CUtensorMap tmk,
+                  const __grid_constant__ CUtensorMap tmv) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle atoms
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int w = blockIdx.x * kWarps + warp;
+  const int W = prm.plan.workers;
+  if (w >= W) return;
+
+  using T = Tile<KV>;
+  uint8_t* ring_ptr = smem + warp * T::kRingBytes;
+  const uint32_t ring = dev::smem_u32(ring_ptr);
+  const uint32_t bars = dev::smem_u32(smem + kWarps * T::kRingBytes) + warp * T::kStages * 8;
+  if (lane == 0) {
+    dev::tma_prefetch_desc(&tmk);
+    dev::tma_prefetch_desc(&tmv);
+    for (int s = 0; s < T::kStages; ++s) dev::mbar_init(bars + s * 8, 1);
+    dev::fence_mbar_init();
+  }
+  __syncwarp();
+
+  const int64_t g0 = worker_start(prm.total, w, W);
+  const int64_t g1 = worker_start(prm.total, w + 1, W);
+  Producer<KV> prod;
+  prod.init(prm, g0, g1, w);
+#pragma unroll 1
+  for (int k = 0; k < T::kStages; ++k) prod.issue(prm, &tmk, &tmv, ring, bars, w, lane);
+
+  PathFor<KV, ACT, G> path;
+  int64_t cg = g0;
+  bool first = true;
+  uint32_t consumed = 0;
+  bool failed = false;
+#pragma unroll 1
+  while (!failed) {
+    const Seg s = next_seg(prm, cg, g1, w, first);
+    first = false;
+    if (!s.valid) break;
+    path.begin(prm, s, lane);
+#pragma unroll 1
+    for (int b = s.b0; b < s.b1; ++b) {
+      const uint32_t stage = consumed % T::kStages;
+      const uint32_t parity = (consumed / T::kStages) & 1u;
+      if (!dev::mbar_wait_bounded(bars + stage * 8, parity, kWaitLimit)) {
+        if (lane == 0) atomicOr(prm.err, kErrTimeout);
+        failed = true;
+        break;
+      }
+      const int nvalid = min(kBlock, s.len - b * kBlock);
+      uint8_t* st = ring_ptr + stage * T::kStageBytes;
+      if (nvalid < kBlock) zero_tail_rows<KV>(st + T::kBytes, nvalid, lane);
+      path.block(ring + stage * T::kStageBytes, ring + stage * T::kStageBytes + T::kBytes, nvalid,
+                 lane);
+      __syncwarp();
+      ++consumed;
+      prod.issue(prm, &tmk, &tmv, ring, bars, w, lane);
+    }
+    if (failed) break;
+    path.finish(prm, s, lane);
+  }
+  if (failed) {
+    // Let copies already in flight land before the CTA's shared memory goes away.
+    for (uint32_t c = consumed; c < prod.issued; ++c)
+      dev::mbar_wait_bounded(bars + (c % T::kStages) * 8, (c / T::kStages) & 1u, kWaitLimit);
+  }
+}
+
+// ===================================================================== reduce
+struct ReduceKParams {
+  uint8_t* out;
+  const float* partials;
+  int64_t q_item_stride;
+  int32_t group;
+  int64_t total;
+  DecodePlan plan;
+};
+
+// Merge the partial slots of one (item, head) into the output.
+template <int ACT, class SlotFn>
+__device__ __forceinline__ void merge_unit(const ReduceKParams& prm, int item, int h, int nslots,
+                                           SlotFn slot_of) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int gg = warp; gg < prm.group; gg += blockDim.x >> 5) {
+    float M = -INFINITY;
+    for (int k = 0; k < nslots; ++k) {
+      const float* ml = prm.partials + static_cast<int64_t>(slot_of(k)) * kPartialSlotFloats +
+                        kMaxGroup * kHeadDim;
+      M = fmaxf(M, ml[2 * gg]);
+    }
+    float L = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < nslots; ++k) {
+      const float* slot = prm.partials + static_cast<int64_t>(slot_of(k)) * kPartialSlotFloats;
+      const float* ml = slot + kMaxGroup * kHeadDim;
+      const float wgt = dev::exp2_approx(ml[2 * gg] - M);
+      L += wgt * ml[2 * gg + 1];
+      const float4 x = reinterpret_cast<const float4*>(slot + gg * kHeadDim)[lane];
+      o.x += wgt * x.x;
+      o.y += wgt * x.y;
+      o.z += wgt * x.z;
+      o.w += wgt * x.w;
+    }
+    const float inv = 1.f / L;
+    uint16_t* orow = reinterpret_cast<uint16_t*>(prm.out) + item * prm.q_item_stride +
+                     (h * prm.group + gg) * kHeadDim + 4 * lane;
+    const uint32_t a = static_cast<uint32_t>(f32_to_act<ACT>(o.x * inv)) |
+                       (static_cast<uint32_t>(f32_to_act<ACT>(o.y * inv)) << 16);
+    const uint32_t b = static_cast<uint32_t>(f32_to_act<ACT>(o.z * inv)) |
+                       (static_cast<uint32_t>(f32_to_act<ACT>(o.w * inv)) << 16);
+    *reinterpret_cast<uint2*>(orow) = make_uint2(a, b);
+  }
+}
+
+// Stream-K: CTA k-1 looks at the boundary between workers k-1 and k and merges
+// the unit that boundary cuts, if it is the first boundary inside that unit.
+template <int ACT>
+__global__ void __launch_bounds__(128) reduce_streamk_kernel(const __grid_constant__ ReduceKParams prm) {
+  const DecodePlan& P = prm.plan;
+  const int W = P.workers;
+  const int k = blockIdx.x + 1;
+  const int64_t bnd = worker_start(prm.total, k, W);
+  const int h = static_cast<int>(bnd / P.per_head);
+  const int64_t r = bnd - static_cast<int64_t>(h) * P.per_head;
+  const int i = find_item(P, r);
+  const int64_t u0 = static_cast<int64_t>(h) * P.per_head + P.pre[i];
+  const int64_t u1 = u0 + (P.pre[i + 1] - P.pre[i]);
+  if (bnd == u0) return;                                   // boundary at a unit start
+  const int64_t prev = worker_start(prm.total, k - 1, W);
+  if (prev > u0) return;                                   // an earlier boundary merges it
+  int last = k;
+  while (last + 1 < W && worker_start(prm.total, last + 1, W) < u1) ++last;
+  const int nslots = last - (k - 1) + 1;
+  const bool prev_first = prev == u0;
+  merge_unit<ACT>(prm, i, h, nslots, [&](int q) {
+    const int wk = k - 1 + q;
+    if (q == 0) return prev_first ? 2 * wk : 2 * wk + 1;
+    return 2 * wk;
+  });
+}
+
+// Fixed partitions: CTA = (head, item); merges the item's partitions if > 1.
+template <int ACT>
+__global__ void __launch_bounds__(128) reduce_fixed_kernel(const __grid_constant__ ReduceKParams prm) {
+  const DecodePlan& P = prm.plan;
+  const int h = blockIdx.x / P.n;
+  const int i = blockIdx.x - h * P.n;
+  const int np = P.pre[i + 1] - P.pre[i];
+  if (np <= 1) return;
+  const int64_t base = static_cast<int64_t>(h) * P.per_head + P.pre[i];
+  merge_unit<ACT>(prm, i, h, np, [&](int q) { return static_cast<int>(base + q); });
+}
+
+// ================================================================== launchers
+template <int KV>
+constexpr size_t smem_bytes() {
+  return 1024 + kWarps * Tile<KV>::kRingBytes + kWarps * Tile<KV>::kStages * 8;
+}
+
+template <int KV, int ACT, int G>
+cudaError_t run_decode(const DecodeKParams& prm, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                       cudaStream_t stream) {
+  constexpr size_t smem = smem_bytes<KV>();
+  static uint64_t configured = 0;  // bit per device: dynamic shared memory attribute set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !(configured >> dev & 1u)) {
+    e = cudaFuncSetAttribute(decode_kernel<KV, ACT, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    if (dev < 64) configured |= uint64_t{1} << dev;
+  }
+  const int grid = (prm.plan.workers + kWarps - 1) / kWarps;
+  decode_kernel<KV, ACT, G><<<grid, kWarps * 32, smem, stream>>>(prm, *tmk, *tmv);
+  return cudaGetLastError();
+}
+
+template <int KV, int ACT>
+cudaError_t dispatch_group(const DecodeKParams& prm, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                           cudaStream_t stream) {
+  switch (prm.group) {
+    case 1: return run_decode<KV, ACT, 1>(prm, tmk, tmv, stream);
+    case 2: return run_decode<KV, ACT, 2>(prm, tmk, tmv, stream);
+    case 4: return run_decode<KV, ACT, 4>(prm, tmk, tmv, stream);
+    case 8: return run_decode<KV, ACT, 8>(prm, tmk, tmv, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+int decode_warps_per_cta() { return kWarps; }
+
+int decode_worker_capacity(int kv_dtype, int /*group*/, int num_sms) {
+  const size_t smem = kv_dtype == kFP8 ? smem_bytes<kFP8>() : smem_bytes<kBF16>();
+  const size_t per_sm = 227 * 1024;
+  const int ctas = std::max<int>(1, static_cast<int>(per_sm / smem));
+  return std::min(kMaxWorkers, num_sms * ctas * kWarps);
+}
+
+cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                          const DecodePlan& plan, const DecodeArgs& args, cudaStream_t stream,
+                          int* launches) {
+  DecodeKParams prm;
+  prm.q = static_cast<const uint8_t*>(args.q);
+  prm.out = static_cast<uint8_t*>(args.out);
+  prm.tables = pool.tables;
+  prm.lens = pool.lens;
+  prm.partials = pool.partials;
+  prm.err = pool.err;
+  prm.k_scale = pool.k_scale;
+  prm.v_scale = pool.v_scale;
+  prm.q_item_stride = args.q_item_stride;
+  prm.scale = args.scale;
+  prm.layer = args.layer;
+  prm.num_kv_heads = pool.num_kv_heads;
+  prm.num_blocks = pool.num_blocks;
+  prm.mbps = pool.mbps;
+  prm.group = args.group;
+  prm.total = plan.per_head * pool.num_kv_heads;
+  std::memcpy(&prm.plan, &plan, sizeof(DecodePlan));
+  // q / out of this launch start at item_offset
+  prm.q += static_cast<int64_t>(args.item_offset) * args.q_item_stride * 2;
+  prm.out += static_cast<int64_t>(args.item_offset) * args.q_item_stride * 2;
+
+  cudaError_t e;
+  if (pool.kv_dtype == kFP8) {
+    e = pool.act_dtype == kBF16 ? dispatch_group<kFP8, kBF16>(prm, tmk, tmv, stream)
+                                : dispatch_group<kFP8, kFP16>(prm, tmk, tmv, stream);
+  } else if (pool.kv_dtype == kBF16) {
+    e = dispatch_group<kBF16, kBF16>(prm, tmk, tmv, stream);
+  } else {
+    e = dispatch_group<kFP16, kFP16>(prm, tmk, tmv, stream);
+  }
+  if (e != cudaSuccess) return e;
+  ++*launches;
+
+  const bool need_reduce =
+      (plan.mode == kSplitStreamK && plan.workers > 1) || plan.mode == kSplitFixed;
+  if (!need_reduce) return cudaSuccess;
+  ReduceKParams rp;
+  rp.out = prm.out;
+  rp.partials = pool.partials;
+  rp.q_item_stride = args.q_item_stride;
+  rp.group = args.group;
+  rp.total = prm.total;
+  std::memcpy(&rp.plan, &plan, sizeof(DecodePlan));
+  if (plan.mode == kSplitStreamK) {
+    const int grid = plan.workers - 1;
+    if (pool.act_dtype == kBF16) reduce_streamk_kernel<kBF16><<<grid, 128, 0, stream>>>(rp);
+    else reduce_streamk_kernel<kFP16><<<grid, 128, 0, stream>>>(rp);
+  } else {
+    const int grid = plan.n * pool.num_kv_heads;
+    if (pool.act_dtype == kBF16) reduce_fixed_kernel<kBF16><<<grid, 128, 0, stream>>>(rp);
+    else reduce_fixed_kernel<kFP16><<<grid, 128, 0, stream>>>(rp);
+  }
+  e = cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+}  // namespace pa

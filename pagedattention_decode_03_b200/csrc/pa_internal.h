@@ -1,0 +1,116 @@
+// Interfaces between the C-ABI layer (api.cpp) and the CUDA kernels.
+//
+// Per-launch metadata travels in the kernel parameters (up to ~30 KB), so a
+// decode step needs no host-to-device copy: the block-table deltas of the
+// step ride along with the append (or copy-on-write) launch that precedes the
+// decode, and the decode launch carries its sequence ids and work prefix sums.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace pa {
+
+enum DType : int32_t { kBF16 = 0, kFP16 = 1, kFP8 = 2 };
+
+constexpr int kHeadDim = 128;
+constexpr int kMaxGroup = 8;          // query heads per KV head handled by one warp
+constexpr int kPartialRowFloats = kHeadDim;
+// One split-KV partial slot: o[8][128] unnormalised fp32, then (m, l)[8].
+constexpr int kPartialSlotFloats = kMaxGroup * (kHeadDim + 2);
+constexpr int kMaxWorkers = 2048;     // warps of one decode launch (stream-K slots = 2x)
+
+// Device error word bits (mirrored in pa.h).
+constexpr uint32_t kErrBadBlock = 0x1u;
+constexpr uint32_t kErrBadLen = 0x2u;
+constexpr uint32_t kErrTimeout = 0x4u;
+
+// ---------------------------------------------------------------- pool view
+struct PoolView {
+  void* k_cache;
+  void* v_cache;
+  const float* k_scale;
+  const float* v_scale;
+  const float* k_inv;
+  const float* v_inv;
+  int32_t* meta;        // [tables: max_seqs*mbps][lens: max_seqs]
+  int32_t* tables;      // = meta
+  int32_t* lens;        // = meta + max_seqs*mbps
+  float* partials;      // [slots][kPartialSlotFloats]
+  uint32_t* err;
+  int64_t partial_slots;
+  int32_t num_layers, num_kv_heads, block_size, num_blocks, max_seqs, mbps;
+  int32_t kv_dtype, act_dtype;
+};
+
+// ------------------------------------------------------ metadata payloads
+// One int32 payload array shared by the small launches; each launcher
+// documents its own packing.
+template <int CAP>
+struct Payload {
+  int32_t v[CAP];
+};
+
+constexpr int kPayloadSmall = 512;
+constexpr int kPayloadLarge = 7168;
+
+// ------------------------------------------------------------ launchers
+// Apply `n` deltas (idx[k], val[k]) to pool.meta.
+cudaError_t launch_meta_apply(const PoolView& pool, const int32_t* idx, const int32_t* val,
+                              int n, cudaStream_t stream);
+
+// Copy-on-write: copy the whole (all layers, K and V) physical block
+// src[k] -> dst[k] for k < n; also applies `nd` mirror deltas.
+cudaError_t launch_cow_copy(const PoolView& pool, const int32_t* src, const int32_t* dst, int n,
+                            const int32_t* didx, const int32_t* dval, int nd,
+                            cudaStream_t stream, int* launches);
+
+// Append T rows: slot[t] = block * B + offset; also applies `nd` deltas.
+cudaError_t launch_append(const PoolView& pool, int layer, const int64_t* slots, int T,
+                          const void* k_new, const void* v_new,
+                          const int32_t* didx, const int32_t* dval, int nd,
+                          cudaStream_t stream, int* launches);
+
+// Decode work description, computed on the host from the host block tables.
+enum SplitMode : int32_t { kSplitStreamK = 0, kSplitFixed = 1, kSplitNever = 2 };
+
+constexpr int kDecodeItemsCap = 512;
+
+struct DecodePlan {
+  int32_t n;              // items in this launch (<= kDecodeItemsCap)
+  int32_t mode;           // SplitMode
+  int32_t part_blocks;    // fixed mode: blocks per partition
+  int32_t workers;        // warps that carry work
+  int64_t per_head;       // work units per KV head (Tn / Pn / n)
+  int32_t seq[kDecodeItemsCap];
+  int32_t pre[kDecodeItemsCap + 1];   // prefix of per-item work units
+};
+
+struct DecodeArgs {
+  const void* q;
+  void* out;
+  int32_t layer;
+  int32_t num_q_heads;
+  int32_t group;          // G = num_q_heads / num_kv_heads
+  float scale;            // softmax scale
+  int64_t q_item_stride;  // elements between consecutive items of q / out (num_q_heads*128)
+  int32_t item_offset;    // index of plan item 0 within the caller's arrays
+};
+
+// Number of decode workers (warps) that fit on the device at once.
+int decode_worker_capacity(int kv_dtype, int group, int num_sms);
+int decode_warps_per_cta();
+
+cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                          const DecodePlan& plan, const DecodeArgs& args, cudaStream_t stream,
+                          int* launches);
+
+// Device properties the planner needs (cached per device by the caller).
+struct DeviceInfo {
+  int num_sms = 0;
+  int device = -1;
+};
+
+}  // namespace pa
