@@ -61,6 +61,12 @@ def parse():
     return ap.parse_args()
 
 
+def pool_steps(a):
+    """Decode steps the pool is sized for (same in both arms): the timed run
+    plus the end-to-end run, and never fewer than the workload's 100."""
+    return max(100, 2 * (a.warmup + a.steps))
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -306,6 +312,17 @@ class Runner:
         self.step_idx += 1
 
 
+def reduce_ranks(vals, op, device, world):
+    """Max or sum of per-rank floats over all ranks (identity for one rank)."""
+    if world <= 1:
+        return [float(v) for v in vals]
+    import torch
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(
+        t, op=torch.distributed.ReduceOp.MAX if op == "max" else torch.distributed.ReduceOp.SUM)
+    return [float(x) for x in t.tolist()]
+
+
 def run_ours(a, rank, world, local_rank):
     import torch
     import workloads
@@ -316,8 +333,7 @@ def run_ours(a, rank, world, local_rank):
         _b.build()
     if world > 1:
         torch.distributed.barrier()
-    total_steps = a.warmup + a.steps + (0 if a.no_e2e else a.warmup + a.steps)
-    w = workloads.workload(a.workload, seed=a.seed + rank, steps=total_steps)
+    w = workloads.workload(a.workload, seed=a.seed + rank, steps=pool_steps(a))
     partition = w.partition_tokens if a.partition is None else a.partition
     r = Runner(w, device, partition, a.seed + rank)
     stream_obj = torch.cuda.current_stream(device)
@@ -341,20 +357,21 @@ def run_ours(a, rank, world, local_rank):
     torch.cuda.synchronize(device)
     with ClockSampler(device.index) as clk:
         start.record()
+        h0 = time.perf_counter()
         for i in range(a.steps):
             r.step(stream, dec_events=ev[i])
+        host_ms = (time.perf_counter() - h0) * 1e3   # host time to enqueue the K steps
         end.record()
         torch.cuda.synchronize(device)
     launches = pa.pa_launch_count(r.pool) - launches0
     ms = start.elapsed_time(end)
     dec_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
     bits = pa.pa_check_device_errors(r.pool)
+    # every rank takes the same collectives, errors included
+    ms, bits = reduce_ranks([ms, float(bits)], "max", device, world)
+    total_bytes, = reduce_ranks([float(total_bytes)], "sum", device, world)
     if bits:
-        raise RuntimeError(f"device error bits 0x{bits:x}")
-    tmax = torch.tensor([ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(tmax, op=torch.distributed.ReduceOp.MAX)
-    ms = float(tmax.item())
+        raise RuntimeError(f"device error bits 0x{int(bits):x}")
 
     # ---- end to end: host (pinned) inputs in, output back, every step
     e2e = None
@@ -384,16 +401,14 @@ def run_ours(a, rank, world, local_rank):
             ho.copy_(r.out, non_blocking=True)
         s1.record()
         torch.cuda.synchronize(device)
-        e_ms = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device=device)
-        if world > 1:
-            torch.distributed.all_reduce(e_ms, op=torch.distributed.ReduceOp.MAX)
-        e_ms = float(e_ms.item())
-        e2e = {"value": world * e2e_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e_ms, = reduce_ranks([s0.elapsed_time(s1)], "max", device, world)
+        e2e_bytes, = reduce_ranks([float(e2e_bytes)], "sum", device, world)
+        e2e = {"value": e2e_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel()) * 2,
                "d2h_bytes_per_step": ho.numel() * 2, "ms_per_step": e_ms / a.steps}
 
     peak, peak_src = peaks()
-    value = world * total_bytes / (ms * 1e-3) / 1e9
+    value = total_bytes / (ms * 1e-3) / 1e9          # bytes of all ranks / max time
     dec_mean = statistics.mean(dec_ms)
     achieved = statistics.mean(dec_bytes) / w.num_layers / (dec_mean * 1e-3) / 1e9
     tr = traffic_record(f"{w.name}:decode")
@@ -427,6 +442,7 @@ def run_ours(a, rank, world, local_rank):
         },
         "logical_decode_gbs": round(world * logical / (ms * 1e-3) / 1e9, 1),
         "gpu_launches": int(launches),
+        "host_enqueue_ms_per_step": round(host_ms / a.steps, 4),
         "clocks": clk.summary(),
         "e2e": e2e,
     }
@@ -523,7 +539,7 @@ def _subset(w, seqs):
 
 def run_reference(a):
     import workloads
-    w = workloads.workload(a.workload, seed=a.seed, steps=a.warmup + a.steps)
+    w = workloads.workload(a.workload, seed=a.seed, steps=pool_steps(a))
     partition = w.partition_tokens if a.partition is None else a.partition
     lens0 = w.lens_before_step(0)
     smp = OracleSample(w, lens0)

@@ -34,8 +34,11 @@ pa_status cuda_fail(cudaError_t e, const char* what) {
   return PA_ERR_CUDA;
 }
 
+// Workspace layout: [header: error word | 256 B] [block-table mirror + lengths]
+// [stream-K arrival counters] [split-KV partial slots]
 constexpr size_t kHeaderBytes = 256;
 constexpr size_t kAlign = 256;
+constexpr size_t kCounterBytes = sizeof(int32_t) * pa::kMaxWorkers;
 constexpr int kMinBlocksPerWorker = 4;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -104,6 +107,8 @@ pa_status ensure_device(pa_pool* p, cudaStream_t stream) {
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
   e = cudaMemsetAsync(p->view.err, 0, sizeof(uint32_t), stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(error word)");
+  e = cudaMemsetAsync(p->view.counters, 0, kCounterBytes, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(counters)");
 
   void* fn = nullptr;
   cudaDriverEntryPointQueryResult q;
@@ -215,7 +220,7 @@ size_t pa_workspace_size(const pa_pool_desc* d) {
   if (!d || d->max_seqs <= 0 || d->max_blocks_per_seq <= 0 || d->num_kv_heads <= 0 ||
       d->block_size <= 0)
     return 0;
-  return kHeaderBytes + align_up(static_cast<size_t>(meta_ints(*d)) * 4) +
+  return kHeaderBytes + align_up(static_cast<size_t>(meta_ints(*d)) * 4) + kCounterBytes +
          static_cast<size_t>(partial_slots(*d)) * pa::kPartialSlotFloats * 4;
 }
 
@@ -284,7 +289,9 @@ pa_status pa_pool_create(const pa_pool_desc* d, pa_pool** out) {
     v.meta = reinterpret_cast<int32_t*>(ws + kHeaderBytes);
     v.tables = v.meta;
     v.lens = v.meta + static_cast<int64_t>(d->max_seqs) * d->max_blocks_per_seq;
-    v.partials = reinterpret_cast<float*>(ws + kHeaderBytes + align_up(meta_ints(*d) * 4));
+    v.counters = reinterpret_cast<int32_t*>(ws + kHeaderBytes + align_up(meta_ints(*d) * 4));
+    v.partials = reinterpret_cast<float*>(ws + kHeaderBytes + align_up(meta_ints(*d) * 4) +
+                                          kCounterBytes);
     v.partial_slots = partial_slots(*d);
   }
   v.num_layers = d->num_layers;

@@ -23,9 +23,10 @@
 //     reaches the PV MMA through movmatrix.  G <= 2: fp32 FMAs on CUDA cores.
 //   * Work is spread over all warps of the GPU in equal shares of KV blocks
 //     (stream-K style): a worker's share can start and end inside a sequence;
-//     partial results (running max m, sum l, unnormalised o) are merged by a
-//     small log-sum-exp reduction kernel.  Fixed-size partitions and "never
-//     split" are the two other modes.
+//     partial results (running max m, sum l, unnormalised o) of a cut
+//     sequence are merged by log-sum-exp inside the kernel, by the last of its
+//     workers to finish.  Fixed-size partitions (merged by a separate
+//     reduction kernel) and "never split" are the two other modes.
 //   * FP8 E4M3 KV: tiles are half the bytes; codes are converted to f16 with
 //     the hardware cvt (exact), K's scale is folded into the logit scale and
 //     V's into the output.
@@ -59,6 +60,7 @@ struct DecodeKParams {
   const int32_t* tables;
   const int32_t* lens;
   float* partials;
+  int32_t* counters;       // stream-K arrival counters (zero between launches)
   uint32_t* err;
   const float* k_scale;
   const float* v_scale;
@@ -88,9 +90,16 @@ __device__ __forceinline__ int64_t worker_start(int64_t total, int w, int W) {
   return (total * w) / W;
 }
 
-// Next segment of a worker whose remaining range is [g, g_end).
+// Worker whose share [worker_start(w), worker_start(w+1)) holds position x:
+// the largest w with total*w < (x+1)*W.
+__device__ __forceinline__ int find_worker(int64_t total, int W, int64_t x) {
+  return min(W - 1, static_cast<int>(((x + 1) * W - 1) / total));
+}
+
+// Next segment of worker `w` (whose whole share starts at g0) within the
+// remaining range [g, g_end).
 __device__ __forceinline__ Seg next_seg(const DecodeKParams& prm, int64_t& g, int64_t g_end,
-                                        int w, bool first) {
+                                        int w, int64_t g0) {
   Seg s;
   s.valid = g < g_end;
   if (!s.valid) return s;
@@ -118,7 +127,7 @@ __device__ __forceinline__ Seg next_seg(const DecodeKParams& prm, int64_t& g, in
     const int64_t take = min(static_cast<int64_t>(unit_nb - s.b0), g_end - g);
     s.b1 = s.b0 + static_cast<int32_t>(take);
     const bool whole = s.b0 == 0 && s.b1 == unit_nb;
-    s.dest = whole ? -1 : (first ? 2 * w : 2 * w + 1);
+    s.dest = whole ? -1 : (g == g0 ? 2 * w : 2 * w + 1);
     g += take;
   } else if (P.mode == kSplitFixed) {
     const int32_t p = static_cast<int32_t>(r - P.pre[s.i]);
@@ -140,22 +149,55 @@ __device__ __forceinline__ Seg next_seg(const DecodeKParams& prm, int64_t& g, in
   return s;
 }
 
+// The segments of one worker, in processing order.  Stream-K: a worker's last
+// segment, when it starts inside the worker's share (the head of a sequence
+// cut at the share's end), is processed first, then the share from its start
+// (whose first segment is the tail of a sequence cut at the share's start).
+// Both halves of every cut sequence thus finish early and the merge of their
+// partial results happens off the kernel's critical path.
+struct Cursor {
+  int64_t g, end, g0, glast;
+  int w;
+  bool second;
+
+  __device__ __forceinline__ void init(const DecodeKParams& prm, int64_t s0, int64_t s1, int wk) {
+    g0 = s0;
+    w = wk;
+    glast = s0;
+    const DecodePlan& P = prm.plan;
+    if (P.mode == kSplitStreamK && s1 > s0) {
+      const int64_t x = s1 - 1;
+      const int64_t h = x / P.per_head;
+      const int i = find_item(P, x - h * P.per_head);
+      glast = max(s0, h * P.per_head + P.pre[i]);
+    }
+    g = glast;
+    end = s1;
+    second = false;
+  }
+
+  __device__ __forceinline__ Seg next(const DecodeKParams& prm) {
+    if (g >= end && !second && glast > g0) {
+      second = true;
+      g = g0;
+      end = glast;
+    }
+    return next_seg(prm, g, end, w, g0);
+  }
+};
+
 // ------------------------------------------------------------------ producer
 template <int KV>
 struct Producer {
-  int64_t g, g_end;
+  Cursor cur;
   Seg seg;
   int32_t b;          // next block of seg to fetch
-  bool first;
   int32_t tc_val, tc_base, tc_seq;
   uint32_t issued;
 
   __device__ __forceinline__ void init(const DecodeKParams& prm, int64_t g0, int64_t g1, int w) {
-    g = g0;
-    g_end = g1;
-    first = true;
-    seg = next_seg(prm, g, g_end, w, first);
-    first = false;
+    cur.init(prm, g0, g1, w);
+    seg = cur.next(prm);
     b = seg.b0;
     tc_seq = -1;
     tc_base = 0;
@@ -169,7 +211,7 @@ struct Producer {
                                         int w, int lane) {
     if (!seg.valid) return;
     if (b == seg.b1) {
-      seg = next_seg(prm, g, g_end, w, false);
+      seg = cur.next(prm);
       if (!seg.valid) return;
       b = seg.b0;
     }
@@ -250,6 +292,151 @@ template <int ACT>
 __device__ __forceinline__ uint16_t f32_to_act(float x) {
   if constexpr (ACT == kBF16) return __bfloat16_as_ushort(__float2bfloat16_rn(x));
   else return __half_as_ushort(__float2half_rn(x));
+}
+
+// ================================================================ LSE merge
+// One warp merges query row `gg` over `nslots` partial slots (m, l, o~):
+//   M = max m_k,  L = sum 2^(m_k - M) l_k,  out = sum 2^(m_k - M) o~_k / L.
+// Partials written by other SMs are read through L2 (ld.global.cg).
+template <int ACT, class SlotFn>
+__device__ __forceinline__ void merge_row(const float* partials, uint16_t* orow, int gg, int nslots,
+                                          SlotFn slot_of, int lane) {
+  auto ml_of = [&](int k) {
+    return partials + static_cast<int64_t>(slot_of(k)) * kPartialSlotFloats + kMaxGroup * kHeadDim +
+           2 * gg;
+  };
+  float M = -INFINITY;
+  for (int k = lane; k < nslots; k += 32) M = fmaxf(M, __ldcg(ml_of(k)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k0 = 0; k0 < nslots; k0 += 32) {
+    const int k = k0 + lane;
+    float wk = 0.f;
+    if (k < nslots) {
+      const float* ml = ml_of(k);
+      wk = dev::exp2_approx(__ldcg(ml) - M);
+      L += wk * __ldcg(ml + 1);
+    }
+    const int cnt = min(32, nslots - k0);
+    for (int j = 0; j < cnt; ++j) {
+      const float wj = __shfl_sync(0xffffffffu, wk, j);
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(
+          partials + static_cast<int64_t>(slot_of(k0 + j)) * kPartialSlotFloats + gg * kHeadDim) + lane);
+      acc.x += wj * x.x;
+      acc.y += wj * x.y;
+      acc.z += wj * x.z;
+      acc.w += wj * x.w;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  const float inv = 1.f / L;
+  const uint32_t a = static_cast<uint32_t>(f32_to_act<ACT>(acc.x * inv)) |
+                     (static_cast<uint32_t>(f32_to_act<ACT>(acc.y * inv)) << 16);
+  const uint32_t b = static_cast<uint32_t>(f32_to_act<ACT>(acc.z * inv)) |
+                     (static_cast<uint32_t>(f32_to_act<ACT>(acc.w * inv)) << 16);
+  *reinterpret_cast<uint2*>(orow + 4 * lane) = make_uint2(a, b);
+}
+
+// One warp merges all G query rows of one unit over `nslots` partial slots:
+// lane k % 32 reads the (m, l) pairs of slot k, every lane owns d = 4*lane ..
+// 4*lane+3 of every row; all loads of one slot are issued together.
+template <int ACT, int G, class SlotFn>
+__device__ __forceinline__ void merge_unit_warp(const float* partials, uint16_t* obase, int nslots,
+                                                SlotFn slot_of, int lane) {
+  float M[G], L[G];
+  float4 acc[G];
+#pragma unroll
+  for (int gg = 0; gg < G; ++gg) {
+    M[gg] = -INFINITY;
+    L[gg] = 0.f;
+    acc[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int k = lane; k < nslots; k += 32) {
+    const float* ml = partials + static_cast<int64_t>(slot_of(k)) * kPartialSlotFloats + kMaxGroup * kHeadDim;
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) M[gg] = fmaxf(M[gg], __ldcg(ml + 2 * gg));
+  }
+#pragma unroll
+  for (int gg = 0; gg < G; ++gg)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M[gg] = fmaxf(M[gg], __shfl_xor_sync(0xffffffffu, M[gg], o));
+  for (int k0 = 0; k0 < nslots; k0 += 32) {
+    const int k = k0 + lane;
+    float wv[G];
+    if (k < nslots) {
+      const float* ml = partials + static_cast<int64_t>(slot_of(k)) * kPartialSlotFloats + kMaxGroup * kHeadDim;
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) {
+        wv[gg] = dev::exp2_approx(__ldcg(ml + 2 * gg) - M[gg]);
+        L[gg] += wv[gg] * __ldcg(ml + 2 * gg + 1);
+      }
+    } else {
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) wv[gg] = 0.f;
+    }
+    const int cnt = min(32, nslots - k0);
+#pragma unroll 2
+    for (int j = 0; j < cnt; ++j) {
+      const float* slot = partials + static_cast<int64_t>(slot_of(k0 + j)) * kPartialSlotFloats;
+      float4 x[G];
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg)
+        x[gg] = __ldcg(reinterpret_cast<const float4*>(slot + gg * kHeadDim) + lane);
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) {
+        const float wj = __shfl_sync(0xffffffffu, wv[gg], j);
+        acc[gg].x += wj * x[gg].x;
+        acc[gg].y += wj * x[gg].y;
+        acc[gg].z += wj * x[gg].z;
+        acc[gg].w += wj * x[gg].w;
+      }
+    }
+  }
+#pragma unroll
+  for (int gg = 0; gg < G; ++gg) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L[gg] += __shfl_xor_sync(0xffffffffu, L[gg], o);
+    const float inv = 1.f / L[gg];
+    const uint32_t a = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].x * inv)) |
+                       (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].y * inv)) << 16);
+    const uint32_t b = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].z * inv)) |
+                       (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].w * inv)) << 16);
+    *reinterpret_cast<uint2*>(obase + gg * kHeadDim + 4 * lane) = make_uint2(a, b);
+  }
+}
+
+// Stream-K: after a worker wrote the partial of a cut unit, it counts itself
+// in; the last of the unit's workers merges all of them into the output and
+// re-arms the counter.  (Counter = the unit's first worker, unique per cut unit.)
+template <int ACT, int G>
+__device__ __forceinline__ void settle_partial(const DecodeKParams& prm, const Seg& s, int lane) {
+  const DecodePlan& P = prm.plan;
+  if (P.mode != kSplitStreamK) return;  // fixed partitions: a separate reduce kernel merges
+  const int W = P.workers;
+  const int64_t u0 = static_cast<int64_t>(s.h) * P.per_head + P.pre[s.i];
+  const int64_t u1 = u0 + (P.pre[s.i + 1] - P.pre[s.i]);
+  const int wa = find_worker(prm.total, W, u0);
+  const int wb = find_worker(prm.total, W, u1 - 1);
+  const int nslots = wb - wa + 1;
+  __threadfence();
+  __syncwarp();
+  int old = 0;
+  if (lane == 0) old = atomicAdd(prm.counters + wa, 1);
+  old = __shfl_sync(0xffffffffu, old, 0);
+  if (old != nslots - 1) return;
+  __threadfence();
+  const bool a_first = worker_start(prm.total, wa, W) == u0;
+  auto slot_of = [&](int q) {
+    const int wk = wa + q;
+    return (q == 0 && !a_first) ? 2 * wk + 1 : 2 * wk;
+  };
+  uint16_t* obase = reinterpret_cast<uint16_t*>(prm.out) + s.i * prm.q_item_stride +
+                    (s.h * G) * kHeadDim;
+  merge_unit_warp<ACT, G>(prm.partials, obase, nslots, slot_of, lane);
+  if (lane == 0) atomicExch(prm.counters + wa, 0);
 }
 
 // ============================================================ tensor-core path
@@ -439,6 +626,7 @@ struct MmaPath {
         if (h0 < G) { ml[2 * h0] = m0; ml[2 * h0 + 1] = lt0; }
         if (h1 < G) { ml[2 * h1] = m1; ml[2 * h1 + 1] = lt1; }
       }
+      settle_partial<ACT, G>(prm, s, lane);
     }
   }
 };
@@ -634,14 +822,17 @@ struct FmaPath {
         }
       }
     }
-    if (s.dest >= 0 && lane == 0) {
-      float* ml = prm.partials + static_cast<int64_t>(s.dest) * kPartialSlotFloats +
-                  kMaxGroup * kHeadDim;
+    if (s.dest >= 0) {
+      if (lane == 0) {
+        float* ml = prm.partials + static_cast<int64_t>(s.dest) * kPartialSlotFloats +
+                    kMaxGroup * kHeadDim;
 #pragma unroll
-      for (int gg = 0; gg < G; ++gg) {
-        ml[2 * gg] = m[gg];
-        ml[2 * gg + 1] = l[gg];
+        for (int gg = 0; gg < G; ++gg) {
+          ml[2 * gg] = m[gg];
+          ml[2 * gg + 1] = l[gg];
+        }
       }
+      settle_partial<ACT, G>(prm, s, lane);
     }
   }
 };
@@ -684,14 +875,13 @@ __global__ void __launch_bounds__(kWarps * 32)
   for (int k = 0; k < T::kStages; ++k) prod.issue(prm, &tmk, &tmv, ring, bars, w, lane);
 
   PathFor<KV, ACT, G> path;
-  int64_t cg = g0;
-  bool first = true;
+  Cursor cur;
+  cur.init(prm, g0, g1, w);
   uint32_t consumed = 0;
   bool failed = false;
 #pragma unroll 1
   while (!failed) {
-    const Seg s = next_seg(prm, cg, g1, w, first);
-    first = false;
+    const Seg s = cur.next(prm);
     if (!s.valid) break;
     path.begin(prm, s, lane);
 #pragma unroll 1
@@ -732,70 +922,8 @@ struct ReduceKParams {
   DecodePlan plan;
 };
 
-// Merge the partial slots of one (item, head) into the output.
-template <int ACT, class SlotFn>
-__device__ __forceinline__ void merge_unit(const ReduceKParams& prm, int item, int h, int nslots,
-                                           SlotFn slot_of) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int gg = warp; gg < prm.group; gg += blockDim.x >> 5) {
-    float M = -INFINITY;
-    for (int k = 0; k < nslots; ++k) {
-      const float* ml = prm.partials + static_cast<int64_t>(slot_of(k)) * kPartialSlotFloats +
-                        kMaxGroup * kHeadDim;
-      M = fmaxf(M, ml[2 * gg]);
-    }
-    float L = 0.f;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k = 0; k < nslots; ++k) {
-      const float* slot = prm.partials + static_cast<int64_t>(slot_of(k)) * kPartialSlotFloats;
-      const float* ml = slot + kMaxGroup * kHeadDim;
-      const float wgt = dev::exp2_approx(ml[2 * gg] - M);
-      L += wgt * ml[2 * gg + 1];
-      const float4 x = reinterpret_cast<const float4*>(slot + gg * kHeadDim)[lane];
-      o.x += wgt * x.x;
-      o.y += wgt * x.y;
-      o.z += wgt * x.z;
-      o.w += wgt * x.w;
-    }
-    const float inv = 1.f / L;
-    uint16_t* orow = reinterpret_cast<uint16_t*>(prm.out) + item * prm.q_item_stride +
-                     (h * prm.group + gg) * kHeadDim + 4 * lane;
-    const uint32_t a = static_cast<uint32_t>(f32_to_act<ACT>(o.x * inv)) |
-                       (static_cast<uint32_t>(f32_to_act<ACT>(o.y * inv)) << 16);
-    const uint32_t b = static_cast<uint32_t>(f32_to_act<ACT>(o.z * inv)) |
-                       (static_cast<uint32_t>(f32_to_act<ACT>(o.w * inv)) << 16);
-    *reinterpret_cast<uint2*>(orow) = make_uint2(a, b);
-  }
-}
-
-// Stream-K: CTA k-1 looks at the boundary between workers k-1 and k and merges
-// the unit that boundary cuts, if it is the first boundary inside that unit.
-template <int ACT>
-__global__ void __launch_bounds__(128) reduce_streamk_kernel(const __grid_constant__ ReduceKParams prm) {
-  const DecodePlan& P = prm.plan;
-  const int W = P.workers;
-  const int k = blockIdx.x + 1;
-  const int64_t bnd = worker_start(prm.total, k, W);
-  const int h = static_cast<int>(bnd / P.per_head);
-  const int64_t r = bnd - static_cast<int64_t>(h) * P.per_head;
-  const int i = find_item(P, r);
-  const int64_t u0 = static_cast<int64_t>(h) * P.per_head + P.pre[i];
-  const int64_t u1 = u0 + (P.pre[i + 1] - P.pre[i]);
-  if (bnd == u0) return;                                   // boundary at a unit start
-  const int64_t prev = worker_start(prm.total, k - 1, W);
-  if (prev > u0) return;                                   // an earlier boundary merges it
-  int last = k;
-  while (last + 1 < W && worker_start(prm.total, last + 1, W) < u1) ++last;
-  const int nslots = last - (k - 1) + 1;
-  const bool prev_first = prev == u0;
-  merge_unit<ACT>(prm, i, h, nslots, [&](int q) {
-    const int wk = k - 1 + q;
-    if (q == 0) return prev_first ? 2 * wk : 2 * wk + 1;
-    return 2 * wk;
-  });
-}
-
-// Fixed partitions: CTA = (head, item); merges the item's partitions if > 1.
+// Fixed partitions: CTA = (head, item); each warp merges query rows of the
+// item's partitions (if there is more than one) into the output.
 template <int ACT>
 __global__ void __launch_bounds__(128) reduce_fixed_kernel(const __grid_constant__ ReduceKParams prm) {
   const DecodePlan& P = prm.plan;
@@ -804,7 +932,12 @@ __global__ void __launch_bounds__(128) reduce_fixed_kernel(const __grid_constant
   const int np = P.pre[i + 1] - P.pre[i];
   if (np <= 1) return;
   const int64_t base = static_cast<int64_t>(h) * P.per_head + P.pre[i];
-  merge_unit<ACT>(prm, i, h, np, [&](int q) { return static_cast<int>(base + q); });
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint16_t* obase = reinterpret_cast<uint16_t*>(prm.out) + i * prm.q_item_stride +
+                    (h * prm.group) * kHeadDim;
+  for (int gg = warp; gg < prm.group; gg += blockDim.x >> 5)
+    merge_row<ACT>(prm.partials, obase + gg * kHeadDim, gg, np,
+                   [&](int q) { return static_cast<int>(base + q); }, lane);
 }
 
 // ================================================================== launchers
@@ -864,6 +997,7 @@ cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CU
   prm.tables = pool.tables;
   prm.lens = pool.lens;
   prm.partials = pool.partials;
+  prm.counters = pool.counters;
   prm.err = pool.err;
   prm.k_scale = pool.k_scale;
   prm.v_scale = pool.v_scale;
@@ -892,9 +1026,9 @@ cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CU
   if (e != cudaSuccess) return e;
   ++*launches;
 
-  const bool need_reduce =
-      (plan.mode == kSplitStreamK && plan.workers > 1) || plan.mode == kSplitFixed;
-  if (!need_reduce) return cudaSuccess;
+  // Stream-K splits are merged inside the decode kernel by the last worker of
+  // each cut unit; fixed partitions get the separate reduction kernel.
+  if (plan.mode != kSplitFixed) return cudaSuccess;
   ReduceKParams rp;
   rp.out = prm.out;
   rp.partials = pool.partials;
@@ -902,15 +1036,9 @@ cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CU
   rp.group = args.group;
   rp.total = prm.total;
   std::memcpy(&rp.plan, &plan, sizeof(DecodePlan));
-  if (plan.mode == kSplitStreamK) {
-    const int grid = plan.workers - 1;
-    if (pool.act_dtype == kBF16) reduce_streamk_kernel<kBF16><<<grid, 128, 0, stream>>>(rp);
-    else reduce_streamk_kernel<kFP16><<<grid, 128, 0, stream>>>(rp);
-  } else {
-    const int grid = plan.n * pool.num_kv_heads;
-    if (pool.act_dtype == kBF16) reduce_fixed_kernel<kBF16><<<grid, 128, 0, stream>>>(rp);
-    else reduce_fixed_kernel<kFP16><<<grid, 128, 0, stream>>>(rp);
-  }
+  const int grid = plan.n * pool.num_kv_heads;
+  if (pool.act_dtype == kBF16) reduce_fixed_kernel<kBF16><<<grid, 128, 0, stream>>>(rp);
+  else reduce_fixed_kernel<kFP16><<<grid, 128, 0, stream>>>(rp);
   e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
   return e;

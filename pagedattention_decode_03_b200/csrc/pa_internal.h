@@ -39,6 +39,7 @@ struct PoolView {
   int32_t* tables;      // = meta
   int32_t* lens;        // = meta + max_seqs*mbps
   float* partials;      // [slots][kPartialSlotFloats]
+  int32_t* counters;    // [kMaxWorkers] stream-K arrival counters, zero between launches
   uint32_t* err;
   int64_t partial_slots;
   int32_t num_layers, num_kv_heads, block_size, num_blocks, max_seqs, mbps;

@@ -38,8 +38,11 @@ class Pair:
     """A GPU pool and an oracle built from the same workload description."""
 
     def __init__(self, w, *, layers=None, num_blocks=None, free_order=None, min_partition=0,
-                 scales_steps=None):
+                 scales_steps=None, oracle_seqs=None):
         self.w = w
+        # sequences whose cache contents the oracle keeps (all by default); the
+        # oracle's pool metadata always follows every sequence
+        self.oracle_seqs = None if oracle_seqs is None else set(oracle_seqs)
         nb = num_blocks or w.num_blocks
         order = w.free_order() if free_order is None else np.asarray(free_order)
         if len(order) != nb:
@@ -72,6 +75,13 @@ class Pair:
             ki = vi = None
             if self.scales is not None:
                 ki, vi = self.scales[2], self.scales[3]
+            if self.oracle_seqs is not None:
+                keep = [t for t, s in enumerate(seqs) if s in self.oracle_seqs]
+                if not keep:
+                    return
+                seqs = [seqs[t] for t in keep]
+                positions = [positions[t] for t in keep]
+                k_bits, v_bits = k_bits[keep], v_bits[keep]
             st = self.oracle.append(layer, seqs, positions, k_bits, v_bits, self.w.act_dtype, ki, vi)
             assert st is Status.OK, st
 
@@ -154,9 +164,14 @@ class Pair:
             assert np.array_equal(gk, o.k[layer][blk, :, t % o.B, :]), ("K", layer, s)
             assert np.array_equal(gv, o.v[layer][blk, :, t % o.B, :]), ("V", layer, s)
 
-    def check_attention(self, layer, seqs, q_bits, out, tol=None):
-        ref = self.oracle_attention(layer, seqs, q_bits)
+    def check_attention(self, layer, seqs, q_bits, out, tol=None, only=None):
+        """Compare the decode output of items `only` (all by default)."""
         got = bits_to_f64(from_dev(out), self.w.act_dtype)
+        if only is not None:
+            seqs = [seqs[i] for i in only]
+            q_bits = q_bits[list(only)]
+            got = got[list(only)]
+        ref = self.oracle_attention(layer, seqs, q_bits)
         err = np.abs(got - ref)
         tol = TOL[self.w.kv_dtype] if tol is None else tol
         assert np.isfinite(got).all()

@@ -311,3 +311,61 @@ def test_errors_leave_state_unchanged():
     with pytest.raises(pa.PAError):
         pa.pa_decode_attention(p.pool, 0, [0], q, torch.empty_like(q), 0.1)   # G = 3
     assert before == (pa.pa_get_free_list(p.pool), pa.pa_get_refcounts(p.pool))
+
+
+@pytest.mark.parametrize("partition", [512, 0, -1])
+def test_fp8_long_context_reduced(partition):
+    """FP8-E4M3 KV with per-(layer, head) scales, 64 q / 8 KV heads, 8 sequences
+    (2,048 tokens here; the full 32,768 below), split-KV partitions + reduce."""
+    w = workload("fp8_long", tokens=2048)
+    p = Pair(w)
+    p.prefill()
+    seqs, pos = p.reserve_step(0)
+    p.append_step(0, 0, seqs, pos)
+    p.check_metadata()
+    p.check_cache(0)
+    q, out = p.decode(0, 0, seqs, partition)
+    p.check_attention(0, seqs, q, out)
+    assert p.device_errors() == 0
+
+
+def test_fp8_long_context_full_size_sampled():
+    """8 x 32,768 tokens, 512-token partitions (4,096 work units + reduce); the
+    oracle keeps the contents of two sequences and checks all their heads."""
+    w = workload("fp8_long")
+    sample = [0, 5]
+    p = Pair(w, oracle_seqs=sample)
+    p.prefill()
+    seqs, pos = p.reserve_step(0)
+    p.append_step(0, 0, seqs, pos)
+    p.check_metadata()
+    p.check_cache(0, seqs=sample)
+    for part in (512, 0):
+        q, out = p.decode(0, 0, seqs, part)
+        p.check_attention(0, seqs, q, out, only=sample)
+    assert p.device_errors() == 0
+
+
+def test_gqa70b_headroom_sampled_layers():
+    """80 layers, 64 q / 8 KV heads, 47 sequences growing from 825 into block 53
+    on the 2,491-block pool; three layers carry data and are compared at steps
+    1, 8 and 16, layer 0 at every step."""
+    w = workload("gqa70b_headroom")
+    layers = [0, 40, 79]
+    p = Pair(w, layers=layers)
+    p.prefill(gpu_layers=layers)
+    for step in range(w.steps):
+        seqs, pos = p.reserve_step(step)
+        for layer in range(w.num_layers):
+            p.append_step(step, layer, seqs, pos)      # oracle keeps only the compared layers
+            if layer in layers and (layer == 0 or step in (0, 7, 15)):
+                q, out = p.decode(step, layer, seqs, 0)
+                p.check_attention(layer, seqs, q, out)
+            else:
+                p.decode(step, layer, seqs, 0)
+        if step in (0, 7, 15):
+            p.check_metadata()
+            for layer in layers:
+                p.check_cache(layer)
+    assert pa.pa_get_free_list(p.pool) == []
+    assert p.device_errors() == 0
