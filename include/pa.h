@@ -184,6 +184,36 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, int32_t n, const int
                               int32_t num_q_heads, const void *q, void *out, float scale,
                               int32_t partition_tokens, void *stream);
 
+/* Decode attention for callers that cannot allocate device memory -- for
+ * example a plugin or custom-operator interface of a serving engine that
+ * reserves all free HBM for its own KV pool and hands a kernel only its input
+ * and output buffers, or a process under a hard memory cap.  Such callers
+ * cannot provide a pool's workspace.  The pages have no counterpart of this
+ * entry point; it computes the same result as pa_decode_attention with the
+ * library's own work split (partition_tokens = 0).
+ *
+ * No pool is involved: `desc` supplies the shapes, dtypes, device, k_cache /
+ * v_cache and (FP8) k_scale / v_scale; its workspace, inverse scales and
+ * free_order are ignored.  block_tables: device int32 [n][desc->max_blocks_per_seq],
+ * row i = physical block ids of sequence i; seq_lens: host int32 [n], tokens
+ * of each sequence (1 .. max_blocks_per_seq * 16); q / out: device
+ * [n][num_q_heads][128] act_dtype.  Limits: block_size 16, n <= 512.
+ *
+ * Allocates nothing (no cudaMalloc/cudaFree).  Its scratch -- split-KV
+ * partial results, arrival counters, a device copy of seq_lens -- is one
+ * static device array of 12 MiB that every GPU loading the library holds
+ * until the process exits.  The first call on a device looks up that array's
+ * device address (once per device, with the device current); make that first
+ * call before any stream capture.  Every call shares the array and clears
+ * what must start at zero, so calls whose work overlaps on the GPU (other
+ * streams, other host threads) race: serialise them, e.g. on one stream.
+ * Errors: PA_ERR_INVALID_ARG (shapes, pointers, lengths; n above 512),
+ * PA_ERR_CUDA. */
+pa_status pa_decode_attention_noalloc(const pa_pool_desc *desc, int32_t layer, int32_t n,
+                                      const int32_t *block_tables, const int32_t *seq_lens,
+                                      int32_t num_q_heads, const void *q, void *out, float scale,
+                                      void *stream);
+
 /* Drop `seq`: every block's reference count falls by one, and blocks that
  * reach zero go to the tail of the free list in logical-block order ([MKV]
  * Block Tables and Sharing).  Errors: PA_ERR_INVALID_ARG, PA_ERR_NO_SEQ. */

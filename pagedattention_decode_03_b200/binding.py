@@ -38,6 +38,7 @@ EXPORTS = (
     "pa_alloc_blocks_n", "pa_fork_cow", "pa_append_kv", "pa_decode_attention", "pa_free",
     "pa_get_seq", "pa_get_refcounts", "pa_get_free_list", "pa_get_cow_log", "pa_launch_count",
     "pa_check_device_errors", "pa_debug_fail_after", "pa_last_error", "pa_status_string",
+    "pa_decode_attention_noalloc",
 )
 
 
@@ -96,6 +97,8 @@ def lib() -> ctypes.CDLL:
         L.pa_fork_cow.argtypes = [vp, i32, i32]
         L.pa_append_kv.argtypes = [vp, i32, i32, _i32p, _i32p, vp, vp, vp]
         L.pa_decode_attention.argtypes = [vp, i32, i32, _i32p, i32, vp, vp, ctypes.c_float, i32, vp]
+        L.pa_decode_attention_noalloc.argtypes = [ctypes.POINTER(pa_pool_desc), i32, i32, vp, _i32p,
+                                                  i32, vp, vp, ctypes.c_float, vp]
         L.pa_free.argtypes = [vp, i32]
         L.pa_get_seq.argtypes = [vp, i32, _i32p, _i32p, i32, _i32p]
         L.pa_get_refcounts.argtypes = [vp, _i32p, i32]
@@ -110,6 +113,7 @@ def lib() -> ctypes.CDLL:
         L.pa_status_string.argtypes = [i32]
         L.pa_status_string.restype = ctypes.c_char_p
         for name in ("pa_pool_create", "pa_alloc_blocks", "pa_alloc_blocks_n", "pa_fork_cow",
+                     "pa_decode_attention_noalloc",
                      "pa_append_kv", "pa_decode_attention", "pa_free", "pa_get_seq",
                      "pa_get_refcounts", "pa_get_free_list", "pa_get_cow_log",
                      "pa_check_device_errors", "pa_debug_fail_after"):
@@ -302,6 +306,28 @@ def pa_decode_attention(pool: Pool, layer: int, seqs, q, out, scale: float,
     _check(lib().pa_decode_attention(pool.handle, layer, n, _ptr(s), hq, ctypes.c_void_p(qp),
                                      ctypes.c_void_p(op), ctypes.c_float(scale),
                                      partition_tokens, _stream(stream)), "pa_decode_attention")
+
+
+def pa_decode_attention_noalloc(desc: pa_pool_desc, layer: int, block_tables, seq_lens, q, out,
+                                scale: float, stream=None) -> None:
+    """Decode attention without a pool or workspace (see include/pa.h): for
+    callers that cannot allocate device memory.  `block_tables` is a device
+    int32 tensor [n][desc.max_blocks_per_seq]; `seq_lens` host lengths [n]."""
+    import torch
+    lens = _i32(seq_lens)
+    n = len(lens)
+    if (not block_tables.is_cuda or block_tables.dtype != torch.int32 or not block_tables.is_contiguous()
+            or tuple(block_tables.shape) != (n, desc.max_blocks_per_seq)):
+        raise ValueError("block_tables must be a contiguous CUDA int32 tensor [n][max_blocks_per_seq]")
+    act = "bf16" if desc.act_dtype == PA_BF16 else "fp16"
+    hq = q.shape[1] if q.dim() == 3 else -1
+    qp = _dev_tensor(q, "q", n, hq, act)
+    op = _dev_tensor(out, "out", n, hq, act)
+    _check(lib().pa_decode_attention_noalloc(ctypes.byref(desc), layer, n,
+                                             ctypes.c_void_p(block_tables.data_ptr()), _ptr(lens), hq,
+                                             ctypes.c_void_p(qp), ctypes.c_void_p(op),
+                                             ctypes.c_float(scale), _stream(stream)),
+           "pa_decode_attention_noalloc")
 
 
 def pa_get_seq(pool: Pool, seq: int):

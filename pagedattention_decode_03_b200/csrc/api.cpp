@@ -82,6 +82,10 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 }  // namespace
 
+namespace pa {
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+}  // namespace pa
+
 struct pa_pool {
   pa_pool_desc d{};
   std::unique_ptr<pa::BlockManager> bm;

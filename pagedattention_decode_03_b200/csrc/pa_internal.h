@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <string>
 
 namespace pa {
 
@@ -107,6 +108,9 @@ int decode_warps_per_cta();
 cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
                           const DecodePlan& plan, const DecodeArgs& args, cudaStream_t stream,
                           int* launches);
+
+// Thread-local text returned by pa_last_error() (defined in api.cpp).
+void set_last_error(const std::string& msg);
 
 // Device properties the planner needs (cached per device by the caller).
 struct DeviceInfo {
