@@ -436,7 +436,11 @@ def run_ours(a, rank, world, local_rank):
             "peak_source": peak_src,
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
-            "traffic": tr["dram_bytes_per_launch"] if tr else None,
+            # ncu dram read+write of one captured launch of this kernel, scaled to this
+            # launch's algorithmic bytes (same workload, a few tokens shorter)
+            "traffic": (int(tr["ratio_to_algorithmic"] * statistics.mean(dec_bytes) / w.num_layers)
+                        if tr else None),
+            "traffic_over_algorithmic": tr["ratio_to_algorithmic"] if tr else None,
             "algorithmic_bytes_per_launch": int(statistics.mean(dec_bytes) / w.num_layers),
             "launch_ms": round(dec_mean, 5),
         },
