@@ -200,7 +200,7 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, int32_t n, const int
  * [n][num_q_heads][128] act_dtype.  Limits: block_size 16, n <= 512.
  *
  * Allocates nothing (no cudaMalloc/cudaFree).  Its scratch -- split-KV
- * partial results, arrival counters, a device copy of seq_lens -- is one
+ * partial results, arrival counters and an error word -- is one
  * static device array of 12 MiB that every GPU loading the library holds
  * until the process exits.  The first call on a device looks up that array's
  * device address (once per device, with the device current); make that first

@@ -454,9 +454,11 @@ pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_
       if (mode == pa::kSplitFixed) units = (nb + part_blocks - 1) / part_blocks;
       if (mode == pa::kSplitNever) units = 1;
       if (mode == pa::kSplitFixed && cnt > 0 && (work + units) * H > slots_cap) break;
+      if (cnt > 0 && (work + units) * H >= (int64_t{1} << 30)) break;  // device positions are int32
       if (mode == pa::kSplitFixed && units * H > slots_cap)
         return fail(PA_ERR_INVALID_ARG, "partition_tokens too small for the workspace");
       plan.seq[cnt] = seqs[at + cnt];
+      plan.len[cnt] = len;
       work += units;
       plan.pre[cnt + 1] = static_cast<int32_t>(work);
       ++cnt;
@@ -549,6 +551,11 @@ pa_status pa_check_device_errors(pa_pool* p, void* stream, uint32_t* bits) {
   if (e != cudaSuccess) return cuda_fail(e, "read error word");
   e = cudaMemset(p->view.err, 0, sizeof(v));
   if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+  if (v & PA_DEVERR_TIMEOUT) {
+    // a worker that gave up may have left a stream-K arrival counter raised
+    e = cudaMemset(p->view.counters, 0, kCounterBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "clear counters");
+  }
   *bits = v;
   if (v) {
     char buf[96];

@@ -58,7 +58,6 @@ struct DecodeKParams {
   const uint8_t* q;
   uint8_t* out;
   const int32_t* tables;
-  const int32_t* lens;
   float* partials;
   int32_t* counters;       // stream-K arrival counters (zero between launches)
   uint32_t* err;
@@ -113,7 +112,7 @@ __device__ __forceinline__ Seg next_seg(const DecodeKParams& prm, int64_t& g, in
     s.i = find_item(P, r);
   }
   s.seq = P.seq[s.i];
-  s.len = prm.lens[s.seq];
+  s.len = P.len[s.i];
   int32_t nb = (s.len + kBlock - 1) / kBlock;
   if (s.len <= 0 || nb > prm.mbps) {
     atomicOr(prm.err, kErrBadLen);
@@ -340,12 +339,17 @@ __device__ __forceinline__ void merge_row(const float* partials, uint16_t* orow,
   *reinterpret_cast<uint2*>(orow + 4 * lane) = make_uint2(a, b);
 }
 
-// One warp merges all G query rows of one unit over `nslots` partial slots:
-// lane k % 32 reads the (m, l) pairs of slot k, every lane owns d = 4*lane ..
-// 4*lane+3 of every row; all loads of one slot are issued together.
+// One warp merges all G query rows of one unit over `nslots` partial slots,
+// online: for each slot k (m_k, l_k, o~_k) the running (M, L, acc) become
+//   M' = max(M, m_k), L' = L 2^(M-M') + l_k 2^(m_k-M'), acc' likewise.
+// Slots are taken a few at a time with every load of a batch issued before
+// any use, so a typical cut sequence (2-4 partials) costs one L2 round trip.
+// Each lane owns d = 4*lane .. 4*lane+3 of every row and reads the (m, l)
+// pairs itself (same address in all lanes: one broadcast transaction).
 template <int ACT, int G, class SlotFn>
 __device__ __forceinline__ void merge_unit_warp(const float* partials, uint16_t* obase, int nslots,
                                                 SlotFn slot_of, int lane) {
+  constexpr int kBatch = G >= 8 ? 2 : (G >= 4 ? 3 : 4);  // loads in flight within the register budget
   float M[G], L[G];
   float4 acc[G];
 #pragma unroll
@@ -354,51 +358,40 @@ __device__ __forceinline__ void merge_unit_warp(const float* partials, uint16_t*
     L[gg] = 0.f;
     acc[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  for (int k = lane; k < nslots; k += 32) {
-    const float* ml = partials + static_cast<int64_t>(slot_of(k)) * kPartialSlotFloats + kMaxGroup * kHeadDim;
+  for (int k0 = 0; k0 < nslots; k0 += kBatch) {
+    float2 ml[kBatch][G];
+    float4 x[kBatch][G];
 #pragma unroll
-    for (int gg = 0; gg < G; ++gg) M[gg] = fmaxf(M[gg], __ldcg(ml + 2 * gg));
-  }
+    for (int j = 0; j < kBatch; ++j) {
+      if (k0 + j < nslots) {
+        const float* slot = partials + static_cast<int64_t>(slot_of(k0 + j)) * kPartialSlotFloats;
 #pragma unroll
-  for (int gg = 0; gg < G; ++gg)
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M[gg] = fmaxf(M[gg], __shfl_xor_sync(0xffffffffu, M[gg], o));
-  for (int k0 = 0; k0 < nslots; k0 += 32) {
-    const int k = k0 + lane;
-    float wv[G];
-    if (k < nslots) {
-      const float* ml = partials + static_cast<int64_t>(slot_of(k)) * kPartialSlotFloats + kMaxGroup * kHeadDim;
-#pragma unroll
-      for (int gg = 0; gg < G; ++gg) {
-        wv[gg] = dev::exp2_approx(__ldcg(ml + 2 * gg) - M[gg]);
-        L[gg] += wv[gg] * __ldcg(ml + 2 * gg + 1);
+        for (int gg = 0; gg < G; ++gg) {
+          ml[j][gg] = __ldcg(reinterpret_cast<const float2*>(slot + kMaxGroup * kHeadDim) + gg);
+          x[j][gg] = __ldcg(reinterpret_cast<const float4*>(slot + gg * kHeadDim) + lane);
+        }
       }
-    } else {
-#pragma unroll
-      for (int gg = 0; gg < G; ++gg) wv[gg] = 0.f;
     }
-    const int cnt = min(32, nslots - k0);
-#pragma unroll 2
-    for (int j = 0; j < cnt; ++j) {
-      const float* slot = partials + static_cast<int64_t>(slot_of(k0 + j)) * kPartialSlotFloats;
-      float4 x[G];
 #pragma unroll
-      for (int gg = 0; gg < G; ++gg)
-        x[gg] = __ldcg(reinterpret_cast<const float4*>(slot + gg * kHeadDim) + lane);
+    for (int j = 0; j < kBatch; ++j) {
+      if (k0 + j < nslots) {
 #pragma unroll
-      for (int gg = 0; gg < G; ++gg) {
-        const float wj = __shfl_sync(0xffffffffu, wv[gg], j);
-        acc[gg].x += wj * x[gg].x;
-        acc[gg].y += wj * x[gg].y;
-        acc[gg].z += wj * x[gg].z;
-        acc[gg].w += wj * x[gg].w;
+        for (int gg = 0; gg < G; ++gg) {
+          const float mn = fmaxf(M[gg], ml[j][gg].x);
+          const float a = dev::exp2_approx(M[gg] - mn);        // 0 on the first slot
+          const float b = dev::exp2_approx(ml[j][gg].x - mn);
+          M[gg] = mn;
+          L[gg] = L[gg] * a + ml[j][gg].y * b;
+          acc[gg].x = acc[gg].x * a + x[j][gg].x * b;
+          acc[gg].y = acc[gg].y * a + x[j][gg].y * b;
+          acc[gg].z = acc[gg].z * a + x[j][gg].z * b;
+          acc[gg].w = acc[gg].w * a + x[j][gg].w * b;
+        }
       }
     }
   }
 #pragma unroll
   for (int gg = 0; gg < G; ++gg) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L[gg] += __shfl_xor_sync(0xffffffffu, L[gg], o);
     const float inv = 1.f / L[gg];
     const uint32_t a = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].x * inv)) |
                        (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].y * inv)) << 16);
@@ -406,6 +399,12 @@ __device__ __forceinline__ void merge_unit_warp(const float* partials, uint16_t*
                        (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].w * inv)) << 16);
     *reinterpret_cast<uint2*>(obase + gg * kHeadDim + 4 * lane) = make_uint2(a, b);
   }
+}
+
+__device__ __forceinline__ int atom_add_acq_rel(int32_t* p, int32_t v) {
+  int32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
 
 // Stream-K: after a worker wrote the partial of a cut unit, it counts itself
@@ -421,13 +420,14 @@ __device__ __forceinline__ void settle_partial(const DecodeKParams& prm, const S
   const int wa = find_worker(prm.total, W, u0);
   const int wb = find_worker(prm.total, W, u1 - 1);
   const int nslots = wb - wa + 1;
-  __threadfence();
+  // __syncwarp orders the other lanes' partial writes before lane 0's
+  // release; the acquire half orders the merge's reads after the arrivals.
   __syncwarp();
   int old = 0;
-  if (lane == 0) old = atomicAdd(prm.counters + wa, 1);
+  if (lane == 0) old = atom_add_acq_rel(prm.counters + wa, 1);
   old = __shfl_sync(0xffffffffu, old, 0);
   if (old != nslots - 1) return;
-  __threadfence();
+  __syncwarp();
   const bool a_first = worker_start(prm.total, wa, W) == u0;
   auto slot_of = [&](int q) {
     const int wk = wa + q;
@@ -436,7 +436,8 @@ __device__ __forceinline__ void settle_partial(const DecodeKParams& prm, const S
   uint16_t* obase = reinterpret_cast<uint16_t*>(prm.out) + s.i * prm.q_item_stride +
                     (s.h * G) * kHeadDim;
   merge_unit_warp<ACT, G>(prm.partials, obase, nslots, slot_of, lane);
-  if (lane == 0) atomicExch(prm.counters + wa, 0);
+  // every arrival is in: re-arm the counter for the next launch (no reply needed)
+  if (lane == 0) asm volatile("st.relaxed.gpu.global.s32 [%0], 0;" ::"l"(prm.counters + wa) : "memory");
 }
 
 // ============================================================ tensor-core path
@@ -995,7 +996,6 @@ cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CU
   prm.q = static_cast<const uint8_t*>(args.q);
   prm.out = static_cast<uint8_t*>(args.out);
   prm.tables = pool.tables;
-  prm.lens = pool.lens;
   prm.partials = pool.partials;
   prm.counters = pool.counters;
   prm.err = pool.err;

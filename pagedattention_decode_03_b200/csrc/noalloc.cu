@@ -10,8 +10,9 @@
 //
 // This entry point needs no pool and no workspace.  The caller passes the
 // cache, its own device block tables and the sequence lengths (host) plus q
-// and out; the split-KV scratch -- partial results, arrival counters and a
-// device copy of the lengths -- lives in one file-scope __device__ array of
+// and out (the lengths travel in the launch parameters); the split-KV
+// scratch -- partial results, arrival counters and an error word -- lives in
+// one file-scope __device__ array of
 // kScratchBytes (12 MiB) that every GPU loading this library holds until the
 // process exits.
 #include <cuda.h>
@@ -29,9 +30,8 @@
 namespace {
 
 constexpr size_t kScratchBytes = size_t{12} << 20;
-constexpr size_t kCountersOff = 0;                                        // int32[kMaxWorkers]
-constexpr size_t kLensOff = kCountersOff + sizeof(int32_t) * pa::kMaxWorkers;  // int32[512]
-constexpr size_t kErrOff = kLensOff + sizeof(int32_t) * pa::kDecodeItemsCap;   // uint32
+constexpr size_t kCountersOff = 0;                                          // int32[kMaxWorkers]
+constexpr size_t kErrOff = kCountersOff + sizeof(int32_t) * pa::kMaxWorkers;  // uint32
 constexpr size_t kPartialsOff = kErrOff + 256;
 constexpr int64_t kScratchSlots =
     static_cast<int64_t>((kScratchBytes - kPartialsOff) / (sizeof(float) * pa::kPartialSlotFloats));
@@ -139,9 +139,12 @@ extern "C" pa_status pa_decode_attention_noalloc(const pa_pool_desc* d, int32_t 
       return fail(PA_ERR_INVALID_ARG, "sequence " + std::to_string(i) +
                                           ": length must be in [1, max_blocks_per_seq * 16]");
     plan.seq[i] = i;  // row i of the caller's block tables
+    plan.len[i] = len;
     work += (len + 15) / 16;
     plan.pre[i + 1] = static_cast<int32_t>(work);
   }
+  if (work * d->num_kv_heads >= (int64_t{1} << 30))
+    return fail(PA_ERR_INVALID_ARG, "too many KV blocks for one call (blocks x kv_heads >= 2^30)");
 
   int prev = -1;
   if (cudaGetDevice(&prev) != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice failed");
@@ -185,8 +188,8 @@ extern "C" pa_status pa_decode_attention_noalloc(const pa_pool_desc* d, int32_t 
   v.k_scale = d->k_scale;
   v.v_scale = d->v_scale;
   v.counters = reinterpret_cast<int32_t*>(scratch + kCountersOff);
-  v.lens = reinterpret_cast<int32_t*>(scratch + kLensOff);
-  v.meta = v.lens;
+  v.lens = nullptr;  // the lengths travel in the launch parameters
+  v.meta = nullptr;
   v.err = reinterpret_cast<uint32_t*>(scratch + kErrOff);
   v.partials = reinterpret_cast<float*>(scratch + kPartialsOff);
   v.partial_slots = kScratchSlots;
@@ -201,15 +204,9 @@ extern "C" pa_status pa_decode_attention_noalloc(const pa_pool_desc* d, int32_t 
   v.act_dtype = d->act_dtype;
 
   // The scratch keeps the previous call's contents: the arrival counters and
-  // the error word must start at zero; the lengths are written by a launch
-  // that carries them in its parameters.
-  cudaError_t e = cudaMemsetAsync(scratch + kCountersOff, 0, kLensOff - kCountersOff, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(scratch + kErrOff, 0, sizeof(uint32_t), s);
+  // the error word must start at zero.
+  cudaError_t e = cudaMemsetAsync(scratch + kCountersOff, 0, kPartialsOff - kCountersOff, s);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("cudaMemsetAsync: ") + cudaGetErrorString(e));
-  int32_t idx[pa::kDecodeItemsCap];
-  for (int32_t i = 0; i < n; ++i) idx[i] = i;
-  e = pa::launch_meta_apply(v, idx, seq_lens, n, s);
-  if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("lengths launch: ") + cudaGetErrorString(e));
 
   const int64_t total = work * d->num_kv_heads;
   int64_t W = std::min<int64_t>(pa::decode_worker_capacity(d->kv_dtype, group, sms), total);

@@ -86,7 +86,8 @@ struct DecodePlan {
   int32_t part_blocks;    // fixed mode: blocks per partition
   int32_t workers;        // warps that carry work
   int64_t per_head;       // work units per KV head (Tn / Pn / n)
-  int32_t seq[kDecodeItemsCap];
+  int32_t seq[kDecodeItemsCap];       // table row of each item
+  int32_t len[kDecodeItemsCap];       // tokens of each item
   int32_t pre[kDecodeItemsCap + 1];   // prefix of per-item work units
 };
 
