@@ -61,10 +61,13 @@ def parse():
     return ap.parse_args()
 
 
+DEFAULT_STEPS = {"tiny": 1, "gqa8b": 100, "gqa70b_headroom": 16, "mha7b_share": 64, "fp8_long": 1}
+
+
 def pool_steps(a):
     """Decode steps the pool is sized for (same in both arms): the timed run
-    plus the end-to-end run, and never fewer than the workload's 100."""
-    return max(100, 2 * (a.warmup + a.steps))
+    plus the end-to-end run, and never fewer than the workload's own count."""
+    return max(DEFAULT_STEPS[a.workload], 2 * (a.warmup + a.steps))
 
 
 def peaks():
