@@ -234,6 +234,16 @@ pa_status pa_get_free_list(pa_pool *pool, int32_t *out, int32_t cap, int32_t *n)
 pa_status pa_get_cow_log(pa_pool *pool, int32_t *pairs, int32_t cap, int32_t *n);
 /* Number of kernels this pool has launched since it was created. */
 uint64_t pa_launch_count(const pa_pool *pool);
+/* Work plan of the last pa_decode_attention call on this pool:
+ * *shared_sets = sibling sets whose common prefix was read once (0 unless
+ * partition_tokens was 0), *kv_tiles = (block, KV head) tiles the call reads
+ * from the cache.  Sequences forked from one prompt share the prompt's blocks
+ * by reference count ([MKV] Block Tables and Sharing; [PAS] The bonus:
+ * sharing via copy-on-write); with partition_tokens = 0 the library reads a
+ * run of at least two full blocks that several of the call's sequences share
+ * once for all of them (up to 8 / G sequences per set), so *kv_tiles can be
+ * below the sum over sequences.  Either pointer may be NULL. */
+pa_status pa_last_decode_plan(const pa_pool *pool, int32_t *shared_sets, int64_t *kv_tiles);
 
 /* Synchronise `stream`, read the device error word, clear it, and store the
  * PA_DEVERR_* bits in *bits.  Returns PA_ERR_DEVICE_CHECK if any bit was set,

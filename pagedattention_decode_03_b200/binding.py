@@ -38,7 +38,7 @@ EXPORTS = (
     "pa_alloc_blocks_n", "pa_fork_cow", "pa_append_kv", "pa_decode_attention", "pa_free",
     "pa_get_seq", "pa_get_refcounts", "pa_get_free_list", "pa_get_cow_log", "pa_launch_count",
     "pa_check_device_errors", "pa_debug_fail_after", "pa_last_error", "pa_status_string",
-    "pa_decode_attention_noalloc",
+    "pa_decode_attention_noalloc", "pa_last_decode_plan",
 )
 
 
@@ -106,6 +106,7 @@ def lib() -> ctypes.CDLL:
         L.pa_get_cow_log.argtypes = [vp, _i32p, i32, _i32p]
         L.pa_launch_count.argtypes = [vp]
         L.pa_launch_count.restype = ctypes.c_uint64
+        L.pa_last_decode_plan.argtypes = [vp, _i32p, ctypes.POINTER(ctypes.c_int64)]
         L.pa_check_device_errors.argtypes = [vp, vp, u32p]
         L.pa_debug_fail_after.argtypes = [vp, i32]
         L.pa_last_error.argtypes = []
@@ -365,6 +366,14 @@ def pa_get_cow_log(pool: Pool):
 
 def pa_launch_count(pool: Pool) -> int:
     return int(lib().pa_launch_count(pool.handle))
+
+
+def pa_last_decode_plan(pool: Pool) -> tuple[int, int]:
+    """(sibling sets read once, (block, KV head) tiles read) of the last decode call."""
+    sets, tiles = ctypes.c_int32(), ctypes.c_int64()
+    _check(lib().pa_last_decode_plan(pool.handle, ctypes.byref(sets), ctypes.byref(tiles)),
+           "pa_last_decode_plan")
+    return sets.value, tiles.value
 
 
 def pa_check_device_errors(pool: Pool, stream=None) -> int:

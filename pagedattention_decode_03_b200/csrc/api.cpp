@@ -38,7 +38,6 @@ pa_status cuda_fail(cudaError_t e, const char* what) {
 // [stream-K arrival counters] [split-KV partial slots]
 constexpr size_t kHeaderBytes = 256;
 constexpr size_t kAlign = 256;
-constexpr size_t kCounterBytes = sizeof(int32_t) * pa::kMaxWorkers;
 constexpr int kMinBlocksPerWorker = 4;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -51,6 +50,12 @@ int32_t min_partition(const pa_pool_desc& d) {
   return d.min_partition_tokens > 0 ? d.min_partition_tokens : 512;
 }
 
+// Arrival counters: one per worker (indexed by the first worker of a cut unit).
+size_t counter_bytes(const pa_pool_desc&) {
+  return align_up(static_cast<size_t>(pa::kMaxWorkers) * sizeof(int32_t));
+}
+
+// Partial slots: two per worker (stream-K) or one per partition (fixed partitions).
 int64_t partial_slots(const pa_pool_desc& d) {
   const int64_t max_tokens = static_cast<int64_t>(d.max_blocks_per_seq) * d.block_size;
   const int64_t parts = (max_tokens + min_partition(d) - 1) / min_partition(d);
@@ -100,6 +105,10 @@ struct pa_pool {
   std::vector<pa::CowPair> cows;
   std::vector<int64_t> slots;
   std::vector<int32_t> a, b;
+  std::vector<int32_t> order, set_of;  // sibling planning
+  // plan of the last decode call (pa_last_decode_plan)
+  int32_t last_sets = 0;
+  int64_t last_tiles = 0;
 };
 
 namespace {
@@ -111,7 +120,7 @@ pa_status ensure_device(pa_pool* p, cudaStream_t stream) {
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
   e = cudaMemsetAsync(p->view.err, 0, sizeof(uint32_t), stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(error word)");
-  e = cudaMemsetAsync(p->view.counters, 0, kCounterBytes, stream);
+  e = cudaMemsetAsync(p->view.counters, 0, counter_bytes(p->d), stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(counters)");
 
   void* fn = nullptr;
@@ -216,6 +225,105 @@ pa_status bm_status(pa::Status s, const char* what) {
   }
 }
 
+// Shortest common prefix (in full blocks) that is read once for a sibling set.
+constexpr int kMinShareBlocks = 2;
+
+// Plan that reads the common prefix of sibling sequences once.  Sequences
+// share blocks by reference count after a fork ([MKV] Block Tables and
+// Sharing; [PAS] The bonus: sharing via copy-on-write), so forks of one
+// prompt hold the same physical ids at the start of their tables.  Items are
+// ordered by their tables (lexicographically), and consecutive items form a
+// set while the set's common run of full blocks stays >= kMinShareBlocks and
+// members x group <= 8 (the query rows of one tensor-core tile).  Each
+// member keeps at least its last block to itself, so every shared block is
+// full for every member.  A set is one work unit: the shared run, then each
+// member's own blocks in member order.  Returns false when no set forms;
+// `sp` is then meaningless.
+bool build_sib_plan(const pa_pool* p, const int32_t* seqs, int32_t cnt, int group, int cap,
+                    pa::SibPlan& sp, std::vector<int32_t>& order, std::vector<int32_t>& set_of) {
+  const int H = p->d.num_kv_heads;
+  const int max_members = pa::kMaxGroup / group;
+  if (max_members < 2 || cnt < 2) return false;
+  const pa::BlockManager& bm = *p->bm;
+  auto nb_of = [&](int i) { return (bm.len(seqs[i]) + 15) / 16; };
+  order.clear();
+  for (int i = 0; i < cnt; ++i)
+    if (nb_of(i) > kMinShareBlocks) order.push_back(i);
+  if (order.size() < 2) return false;
+  std::sort(order.begin(), order.end(), [&](int a, int b) {
+    const std::vector<int32_t>& ta = bm.table(seqs[a]);
+    const std::vector<int32_t>& tb = bm.table(seqs[b]);
+    const size_t m = std::min(ta.size(), tb.size());
+    for (size_t k = 0; k < m; ++k)
+      if (ta[k] != tb[k]) return ta[k] < tb[k];
+    return ta.size() != tb.size() ? ta.size() < tb.size() : a < b;
+  });
+  // sets, in sorted order: members order[a .. b), shared run cp
+  set_of.assign(cnt, -1);
+  int nu = 0, placed = 0;
+  int64_t work = 0;
+  sp.pre[0] = 0;
+  sp.mem0[0] = 0;
+  size_t a = 0;
+  while (a < order.size()) {
+    const std::vector<int32_t>& ta = bm.table(seqs[order[a]]);
+    int cp = nb_of(order[a]) - 1;
+    size_t b = a + 1;
+    while (b < order.size() && static_cast<int>(b - a) < max_members) {
+      const std::vector<int32_t>& tb = bm.table(seqs[order[b]]);
+      const int lim = std::min(cp, nb_of(order[b]) - 1);
+      int l = 0;
+      while (l < lim && ta[l] == tb[l]) ++l;
+      if (l < kMinShareBlocks) break;
+      cp = l;
+      ++b;
+    }
+    if (b - a < 2) {
+      ++a;
+      continue;
+    }
+    int64_t pos = cp;
+    for (size_t j = a; j < b; ++j) {
+      const int it = order[j];
+      set_of[it] = nu;
+      sp.mem[placed++] = static_cast<int16_t>(it);
+      sp.part[it] = static_cast<int32_t>(pos);
+      pos += nb_of(it) - cp;
+    }
+    sp.cp[nu] = cp;
+    work += pos;
+    sp.pre[nu + 1] = static_cast<int32_t>(work);
+    sp.mem0[nu + 1] = static_cast<int16_t>(placed);
+    ++nu;
+    a = b;
+  }
+  if (nu == 0) return false;
+  const int sets = nu;
+  for (int i = 0; i < cnt; ++i) {  // every other item is a unit of its own
+    sp.seq[i] = seqs[i];
+    sp.len[i] = bm.len(seqs[i]);
+    if (set_of[i] >= 0) continue;
+    sp.mem[placed++] = static_cast<int16_t>(i);
+    sp.part[i] = 0;
+    sp.cp[nu] = 0;
+    work += nb_of(i);
+    sp.pre[nu + 1] = static_cast<int32_t>(work);
+    sp.mem0[nu + 1] = static_cast<int16_t>(placed);
+    ++nu;
+  }
+  sp.n = cnt;
+  sp.nu = nu;
+  sp.per_head = work;
+  const int64_t total = work * H;
+  if (total >= (int64_t{1} << 30)) return false;
+  int64_t W = std::min<int64_t>(cap, total);
+  W = std::min<int64_t>(W, std::max<int64_t>(1, (total + kMinBlocksPerWorker - 1) / kMinBlocksPerWorker));
+  W = std::min<int64_t>(W, p->view.partial_slots / 2);
+  sp.workers = static_cast<int32_t>(std::max<int64_t>(1, W));
+  sp.sets = sets;
+  return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -224,7 +332,7 @@ size_t pa_workspace_size(const pa_pool_desc* d) {
   if (!d || d->max_seqs <= 0 || d->max_blocks_per_seq <= 0 || d->num_kv_heads <= 0 ||
       d->block_size <= 0)
     return 0;
-  return kHeaderBytes + align_up(static_cast<size_t>(meta_ints(*d)) * 4) + kCounterBytes +
+  return kHeaderBytes + align_up(static_cast<size_t>(meta_ints(*d)) * 4) + counter_bytes(*d) +
          static_cast<size_t>(partial_slots(*d)) * pa::kPartialSlotFloats * 4;
 }
 
@@ -295,7 +403,7 @@ pa_status pa_pool_create(const pa_pool_desc* d, pa_pool** out) {
     v.lens = v.meta + static_cast<int64_t>(d->max_seqs) * d->max_blocks_per_seq;
     v.counters = reinterpret_cast<int32_t*>(ws + kHeaderBytes + align_up(meta_ints(*d) * 4));
     v.partials = reinterpret_cast<float*>(ws + kHeaderBytes + align_up(meta_ints(*d) * 4) +
-                                          kCounterBytes);
+                                          counter_bytes(*d));
     v.partial_slots = partial_slots(*d);
   }
   v.num_layers = d->num_layers;
@@ -419,6 +527,8 @@ pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_
     if (!p->bm->active(seqs[i])) return fail(PA_ERR_NO_SEQ, "pa_decode_attention: no such sequence");
     if (p->bm->len(seqs[i]) < 1) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: empty sequence");
   }
+  p->last_sets = 0;
+  p->last_tiles = 0;
   if (n == 0) return PA_OK;
   DeviceGuard guard(p->d.device);
   if (!guard.ok) return fail(PA_ERR_CUDA, "cannot select the pool's device");
@@ -445,7 +555,7 @@ pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_
     // Items of this launch: up to the parameter capacity, and (fixed mode) the
     // partial slots the workspace holds.
     int32_t cnt = 0;
-    int64_t work = 0;
+    int64_t work = 0, blocks = 0;
     plan.pre[0] = 0;
     while (at + cnt < n && cnt < pa::kDecodeItemsCap) {
       const int32_t len = p->bm->len(seqs[at + cnt]);
@@ -460,6 +570,7 @@ pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_
       plan.seq[cnt] = seqs[at + cnt];
       plan.len[cnt] = len;
       work += units;
+      blocks += nb;
       plan.pre[cnt + 1] = static_cast<int32_t>(work);
       ++cnt;
     }
@@ -476,7 +587,17 @@ pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_
     plan.workers = static_cast<int32_t>(std::max<int64_t>(1, W));
     args.item_offset = at;
     int launches = 0;
-    cudaError_t e = pa::launch_decode(p->view, &p->tmk, &p->tmv, plan, args, s, &launches);
+    cudaError_t e;
+    static thread_local pa::SibPlan sib;
+    if (mode == pa::kSplitStreamK && group <= 4 &&
+        build_sib_plan(p, seqs + at, cnt, group, cap, sib, p->order, p->set_of)) {
+      e = pa::launch_decode_sib(p->view, &p->tmk, &p->tmv, sib, args, s, &launches);
+      p->last_sets += sib.sets;
+      p->last_tiles += sib.per_head * H;
+    } else {
+      e = pa::launch_decode(p->view, &p->tmk, &p->tmv, plan, args, s, &launches);
+      p->last_tiles += blocks * H;
+    }
     p->launches += launches;
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     at += cnt;
@@ -553,7 +674,7 @@ pa_status pa_check_device_errors(pa_pool* p, void* stream, uint32_t* bits) {
   if (e != cudaSuccess) return cuda_fail(e, "clear error word");
   if (v & PA_DEVERR_TIMEOUT) {
     // a worker that gave up may have left a stream-K arrival counter raised
-    e = cudaMemset(p->view.counters, 0, kCounterBytes);
+    e = cudaMemset(p->view.counters, 0, counter_bytes(p->d));
     if (e != cudaSuccess) return cuda_fail(e, "clear counters");
   }
   *bits = v;
@@ -562,6 +683,14 @@ pa_status pa_check_device_errors(pa_pool* p, void* stream, uint32_t* bits) {
     std::snprintf(buf, sizeof(buf), "device check failed: bits 0x%x", v);
     return fail(PA_ERR_DEVICE_CHECK, buf);
   }
+  return PA_OK;
+}
+
+pa_status pa_last_decode_plan(const pa_pool* p, int32_t* shared_sets, int64_t* kv_tiles) {
+  g_last_error.clear();
+  if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
+  if (shared_sets) *shared_sets = p->last_sets;
+  if (kv_tiles) *kv_tiles = p->last_tiles;
   return PA_OK;
 }
 

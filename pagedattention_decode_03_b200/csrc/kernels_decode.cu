@@ -54,6 +54,7 @@ struct Tile {
   static constexpr int kRingBytes = kStages * kStageBytes;
 };
 
+template <class PlanT>
 struct DecodeKParams {
   const uint8_t* q;
   uint8_t* out;
@@ -67,17 +68,38 @@ struct DecodeKParams {
   float scale;
   int32_t layer, num_kv_heads, num_blocks, mbps, group;
   int64_t total;           // work units over all heads
-  DecodePlan plan;
+  PlanT plan;
 };
 
+template <class PlanT>
+constexpr bool kIsSib = std::is_same<PlanT, SibPlan>::value;
+template <class Prm>
+constexpr bool kSibParams = std::is_same<Prm, DecodeKParams<SibPlan>>::value;
+
+// A worker's contiguous piece of one work unit.  Positions b0 .. b1-1 are the
+// unit's KV blocks in order (for a plain unit: table blocks of item i).
 struct Seg {
   int32_t h, i, b0, b1, dest, len, seq;
+  int32_t k;      // work unit (== i for plain plans)
   bool valid;
+  bool shared;    // a sibling set (two or more items) of a sibling plan
 };
 
-// Index of the item whose prefix range holds r: pre[i] <= r < pre[i+1].
-__device__ __forceinline__ int find_item(const DecodePlan& P, int64_t r) {
-  int lo = 0, hi = P.n - 1;
+// Table position, valid length and active query rows of one KV block.
+struct BlockRef {
+  int32_t seq, b, len;
+  uint32_t cols;  // bit r set: query row r takes part (all 8 for plain units)
+};
+
+__device__ __forceinline__ int n_entries(const DecodePlan& P) { return P.n; }
+__device__ __forceinline__ int n_entries(const SibPlan& P) { return P.nu; }
+__device__ __forceinline__ int plan_mode(const DecodePlan& P) { return P.mode; }
+__device__ __forceinline__ int plan_mode(const SibPlan&) { return kSplitStreamK; }
+
+// Index of the entry whose prefix range holds r: pre[i] <= r < pre[i+1].
+template <class PlanT>
+__device__ __forceinline__ int find_item(const PlanT& P, int64_t r) {
+  int lo = 0, hi = n_entries(P) - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (P.pre[mid] <= r) lo = mid; else hi = mid - 1;
@@ -97,10 +119,11 @@ __device__ __forceinline__ int find_worker(int64_t total, int W, int64_t x) {
 
 // Next segment of worker `w` (whose whole share starts at g0) within the
 // remaining range [g, g_end).
-__device__ __forceinline__ Seg next_seg(const DecodeKParams& prm, int64_t& g, int64_t g_end,
-                                        int w, int64_t g0) {
+__device__ __forceinline__ Seg next_seg(const DecodeKParams<DecodePlan>& prm, int64_t& g,
+                                        int64_t g_end, int w, int64_t g0) {
   Seg s;
   s.valid = g < g_end;
+  s.shared = false;
   if (!s.valid) return s;
   const DecodePlan& P = prm.plan;
   const int64_t per_head = P.per_head;
@@ -111,6 +134,7 @@ __device__ __forceinline__ Seg next_seg(const DecodeKParams& prm, int64_t& g, in
   } else {
     s.i = find_item(P, r);
   }
+  s.k = s.i;
   s.seq = P.seq[s.i];
   s.len = P.len[s.i];
   int32_t nb = (s.len + kBlock - 1) / kBlock;
@@ -148,6 +172,59 @@ __device__ __forceinline__ Seg next_seg(const DecodeKParams& prm, int64_t& g, in
   return s;
 }
 
+// Sibling plan (always stream-K): same cutting and partial slots as a plain
+// stream-K plan, over units that may hold several items.
+__device__ __forceinline__ Seg next_seg(const DecodeKParams<SibPlan>& prm, int64_t& g,
+                                        int64_t g_end, int w, int64_t g0) {
+  Seg s;
+  s.valid = g < g_end;
+  if (!s.valid) return s;
+  const SibPlan& P = prm.plan;
+  s.h = static_cast<int32_t>(g / P.per_head);
+  const int64_t r = g - static_cast<int64_t>(s.h) * P.per_head;
+  s.k = find_item(P, r);
+  const int m0 = P.mem0[s.k];
+  s.shared = P.mem0[s.k + 1] - m0 > 1;
+  s.i = P.mem[m0];
+  s.seq = P.seq[s.i];
+  s.len = P.len[s.i];
+  const int32_t unit_nb = P.pre[s.k + 1] - P.pre[s.k];
+  if (!s.shared && (s.len <= 0 || (s.len + kBlock - 1) / kBlock != unit_nb || unit_nb > prm.mbps))
+    atomicOr(prm.err, kErrBadLen);
+  s.b0 = static_cast<int32_t>(r - P.pre[s.k]);
+  const int64_t take = min(static_cast<int64_t>(unit_nb - s.b0), g_end - g);
+  s.b1 = s.b0 + static_cast<int32_t>(take);
+  const bool whole = s.b0 == 0 && s.b1 == unit_nb;
+  s.dest = whole ? -1 : (g == g0 ? 2 * w : 2 * w + 1);
+  g += take;
+  return s;
+}
+
+// Where position o of segment s lives.  Plain plans: block o of the item.
+// Sibling plans: positions below the unit's shared run cp are the common
+// blocks (every row takes part); after it come the members' own blocks in
+// member order, each taken only by that member's G rows.
+template <int G>
+__device__ __forceinline__ BlockRef locate(const DecodeKParams<DecodePlan>&, const Seg& s, int o) {
+  return BlockRef{s.seq, o, s.len, 0xffu};
+}
+template <int G>
+__device__ __forceinline__ BlockRef locate(const DecodeKParams<SibPlan>& prm, const Seg& s, int o) {
+  const SibPlan& P = prm.plan;
+  const int cp = P.cp[s.k];
+  if (o < cp) return BlockRef{s.seq, o, s.len, 0xffu};
+  const int m0 = P.mem0[s.k], m = P.mem0[s.k + 1] - m0;
+  int j = 0, item = s.i;
+  for (int jj = 1; jj < m; ++jj) {
+    const int it = P.mem[m0 + jj];
+    if (P.part[it] > o) break;
+    j = jj;
+    item = it;
+  }
+  return BlockRef{P.seq[item], cp + (o - P.part[item]), P.len[item],
+                  ((1u << G) - 1u) << (j * G)};
+}
+
 // The segments of one worker, in processing order.  Stream-K: a worker's last
 // segment, when it starts inside the worker's share (the head of a sequence
 // cut at the share's end), is processed first, then the share from its start
@@ -159,12 +236,13 @@ struct Cursor {
   int w;
   bool second;
 
-  __device__ __forceinline__ void init(const DecodeKParams& prm, int64_t s0, int64_t s1, int wk) {
+  template <class Prm>
+  __device__ __forceinline__ void init(const Prm& prm, int64_t s0, int64_t s1, int wk) {
     g0 = s0;
     w = wk;
     glast = s0;
-    const DecodePlan& P = prm.plan;
-    if (P.mode == kSplitStreamK && s1 > s0) {
+    const auto& P = prm.plan;
+    if (plan_mode(P) == kSplitStreamK && s1 > s0) {
       const int64_t x = s1 - 1;
       const int64_t h = x / P.per_head;
       const int i = find_item(P, x - h * P.per_head);
@@ -175,7 +253,8 @@ struct Cursor {
     second = false;
   }
 
-  __device__ __forceinline__ Seg next(const DecodeKParams& prm) {
+  template <class Prm>
+  __device__ __forceinline__ Seg next(const Prm& prm) {
     if (g >= end && !second && glast > g0) {
       second = true;
       g = g0;
@@ -194,7 +273,8 @@ struct Producer {
   int32_t tc_val, tc_base, tc_seq;
   uint32_t issued;
 
-  __device__ __forceinline__ void init(const DecodeKParams& prm, int64_t g0, int64_t g1, int w) {
+  template <class Prm>
+  __device__ __forceinline__ void init(const Prm& prm, int64_t g0, int64_t g1, int w) {
     cur.init(prm, g0, g1, w);
     seg = cur.next(prm);
     b = seg.b0;
@@ -205,7 +285,8 @@ struct Producer {
   }
 
   // Fetch the next block of this worker into stage issued % kStages.
-  __device__ __forceinline__ void issue(const DecodeKParams& prm, const CUtensorMap* tmk,
+  template <class Prm>
+  __device__ __forceinline__ void issue(const Prm& prm, const CUtensorMap* tmk,
                                         const CUtensorMap* tmv, uint32_t ring, uint32_t bars,
                                         int w, int lane) {
     if (!seg.valid) return;
@@ -214,13 +295,14 @@ struct Producer {
       if (!seg.valid) return;
       b = seg.b0;
     }
-    if (seg.seq != tc_seq || b < tc_base || b >= tc_base + 32) {
-      tc_seq = seg.seq;
-      tc_base = b;
-      const int idx = b + lane;
-      tc_val = idx < prm.mbps ? prm.tables[static_cast<int64_t>(seg.seq) * prm.mbps + idx] : 0;
+    const BlockRef br = locate<1>(prm, seg, b);
+    if (br.seq != tc_seq || br.b < tc_base || br.b >= tc_base + 32) {
+      tc_seq = br.seq;
+      tc_base = br.b;
+      const int idx = br.b + lane;
+      tc_val = idx >= 0 && idx < prm.mbps ? prm.tables[static_cast<int64_t>(br.seq) * prm.mbps + idx] : 0;
     }
-    int32_t phys = __shfl_sync(0xffffffffu, tc_val, b - tc_base);
+    int32_t phys = __shfl_sync(0xffffffffu, tc_val, br.b - tc_base);
     if (static_cast<uint32_t>(phys) >= static_cast<uint32_t>(prm.num_blocks)) {
       if (lane == 0) atomicOr(prm.err, kErrBadBlock);
       phys = 0;
@@ -339,36 +421,65 @@ __device__ __forceinline__ void merge_row(const float* partials, uint16_t* orow,
   *reinterpret_cast<uint2*>(orow + 4 * lane) = make_uint2(a, b);
 }
 
-// One warp merges all G query rows of one unit over `nslots` partial slots,
-// online: for each slot k (m_k, l_k, o~_k) the running (M, L, acc) become
-//   M' = max(M, m_k), L' = L 2^(M-M') + l_k 2^(m_k-M'), acc' likewise.
+// Query rows of a segment: a plain unit has its item's G query heads of KV
+// head h (rows 0 .. G-1); a sibling set has member j's G heads at rows
+// j*G .. j*G+G-1.  item_of_row(r) is the item whose output row r is.
+template <int G>
+__device__ __forceinline__ int unit_rows(const DecodeKParams<DecodePlan>&, const Seg&) { return G; }
+template <int G>
+__device__ __forceinline__ int unit_rows(const DecodeKParams<SibPlan>& prm, const Seg& s) {
+  return (prm.plan.mem0[s.k + 1] - prm.plan.mem0[s.k]) * G;
+}
+template <int G>
+__device__ __forceinline__ int item_of_row(const DecodeKParams<DecodePlan>&, const Seg& s, int) {
+  return s.i;
+}
+template <int G>
+__device__ __forceinline__ int item_of_row(const DecodeKParams<SibPlan>& prm, const Seg& s, int r) {
+  return prm.plan.mem[prm.plan.mem0[s.k] + r / G];
+}
+// Element offset of (row r, d = 0) in q / out.
+template <int G, class Prm>
+__device__ __forceinline__ int64_t row_offset(const Prm& prm, const Seg& s, int r) {
+  return item_of_row<G>(prm, s, r) * prm.q_item_stride + (s.h * G + r % G) * kHeadDim;
+}
+
+// One warp merges query rows 0 .. rows-1 (rows <= R) of one unit over
+// `nslots` partial slots, online: for each slot k (m_k, l_k, o~_k) the running
+// (M, L, acc) become
+//   M' = max(M, m_k), L' = L 2^(M-M') + l_k 2^(m_k-M'), acc' likewise,
+// with 0 in place of M' while every slot seen so far is empty (m = -inf, a
+// row that no token of those slots reached).
 // Slots are taken a few at a time with every load of a batch issued before
 // any use, so a typical cut sequence (2-4 partials) costs one L2 round trip.
 // Each lane owns d = 4*lane .. 4*lane+3 of every row and reads the (m, l)
 // pairs itself (same address in all lanes: one broadcast transaction).
-template <int ACT, int G, class SlotFn>
-__device__ __forceinline__ void merge_unit_warp(const float* partials, uint16_t* obase, int nslots,
-                                                SlotFn slot_of, int lane) {
-  constexpr int kBatch = G >= 8 ? 2 : (G >= 4 ? 3 : 4);  // loads in flight within the register budget
-  float M[G], L[G];
-  float4 acc[G];
+// out_of(r) = element offset of output row r.
+template <int ACT, int R, class SlotFn, class OutFn>
+__device__ __forceinline__ void merge_unit_warp(const float* partials, uint16_t* out, int nslots,
+                                                int rows, SlotFn slot_of, OutFn out_of, int lane) {
+  constexpr int kBatch = R >= 8 ? 2 : (R >= 4 ? 3 : 4);  // loads in flight within the register budget
+  float M[R], L[R];
+  float4 acc[R];
 #pragma unroll
-  for (int gg = 0; gg < G; ++gg) {
+  for (int gg = 0; gg < R; ++gg) {
     M[gg] = -INFINITY;
     L[gg] = 0.f;
     acc[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   for (int k0 = 0; k0 < nslots; k0 += kBatch) {
-    float2 ml[kBatch][G];
-    float4 x[kBatch][G];
+    float2 ml[kBatch][R];
+    float4 x[kBatch][R];
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
       if (k0 + j < nslots) {
         const float* slot = partials + static_cast<int64_t>(slot_of(k0 + j)) * kPartialSlotFloats;
 #pragma unroll
-        for (int gg = 0; gg < G; ++gg) {
-          ml[j][gg] = __ldcg(reinterpret_cast<const float2*>(slot + kMaxGroup * kHeadDim) + gg);
-          x[j][gg] = __ldcg(reinterpret_cast<const float4*>(slot + gg * kHeadDim) + lane);
+        for (int gg = 0; gg < R; ++gg) {
+          if (gg < rows) {
+            ml[j][gg] = __ldcg(reinterpret_cast<const float2*>(slot + kMaxGroup * kHeadDim) + gg);
+            x[j][gg] = __ldcg(reinterpret_cast<const float4*>(slot + gg * kHeadDim) + lane);
+          }
         }
       }
     }
@@ -376,28 +487,33 @@ __device__ __forceinline__ void merge_unit_warp(const float* partials, uint16_t*
     for (int j = 0; j < kBatch; ++j) {
       if (k0 + j < nslots) {
 #pragma unroll
-        for (int gg = 0; gg < G; ++gg) {
-          const float mn = fmaxf(M[gg], ml[j][gg].x);
-          const float a = dev::exp2_approx(M[gg] - mn);        // 0 on the first slot
-          const float b = dev::exp2_approx(ml[j][gg].x - mn);
-          M[gg] = mn;
-          L[gg] = L[gg] * a + ml[j][gg].y * b;
-          acc[gg].x = acc[gg].x * a + x[j][gg].x * b;
-          acc[gg].y = acc[gg].y * a + x[j][gg].y * b;
-          acc[gg].z = acc[gg].z * a + x[j][gg].z * b;
-          acc[gg].w = acc[gg].w * a + x[j][gg].w * b;
+        for (int gg = 0; gg < R; ++gg) {
+          if (gg < rows) {
+            const float mn = fmaxf(M[gg], ml[j][gg].x);
+            const float ref = mn == -INFINITY ? 0.f : mn;
+            const float a = dev::exp2_approx(M[gg] - ref);        // 0 on the first slot
+            const float b = dev::exp2_approx(ml[j][gg].x - ref);
+            M[gg] = mn;
+            L[gg] = L[gg] * a + ml[j][gg].y * b;
+            acc[gg].x = acc[gg].x * a + x[j][gg].x * b;
+            acc[gg].y = acc[gg].y * a + x[j][gg].y * b;
+            acc[gg].z = acc[gg].z * a + x[j][gg].z * b;
+            acc[gg].w = acc[gg].w * a + x[j][gg].w * b;
+          }
         }
       }
     }
   }
 #pragma unroll
-  for (int gg = 0; gg < G; ++gg) {
-    const float inv = 1.f / L[gg];
-    const uint32_t a = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].x * inv)) |
-                       (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].y * inv)) << 16);
-    const uint32_t b = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].z * inv)) |
-                       (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].w * inv)) << 16);
-    *reinterpret_cast<uint2*>(obase + gg * kHeadDim + 4 * lane) = make_uint2(a, b);
+  for (int gg = 0; gg < R; ++gg) {
+    if (gg < rows) {
+      const float inv = 1.f / L[gg];
+      const uint32_t a = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].x * inv)) |
+                         (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].y * inv)) << 16);
+      const uint32_t b = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].z * inv)) |
+                         (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].w * inv)) << 16);
+      *reinterpret_cast<uint2*>(out + out_of(gg) + 4 * lane) = make_uint2(a, b);
+    }
   }
 }
 
@@ -409,14 +525,15 @@ __device__ __forceinline__ int atom_add_acq_rel(int32_t* p, int32_t v) {
 
 // Stream-K: after a worker wrote the partial of a cut unit, it counts itself
 // in; the last of the unit's workers merges all of them into the output and
-// re-arms the counter.  (Counter = the unit's first worker, unique per cut unit.)
-template <int ACT, int G>
-__device__ __forceinline__ void settle_partial(const DecodeKParams& prm, const Seg& s, int lane) {
-  const DecodePlan& P = prm.plan;
-  if (P.mode != kSplitStreamK) return;  // fixed partitions: a separate reduce kernel merges
+// re-arms the counter.  (Counter = the unit's first worker, unique per cut
+// unit.)  R = row capacity of the merge (rows <= R).
+template <int ACT, int G, int R, class Prm>
+__device__ __forceinline__ void settle_partial(const Prm& prm, const Seg& s, int rows, int lane) {
+  const auto& P = prm.plan;
+  if (plan_mode(P) != kSplitStreamK) return;  // fixed partitions: a separate reduce kernel merges
   const int W = P.workers;
-  const int64_t u0 = static_cast<int64_t>(s.h) * P.per_head + P.pre[s.i];
-  const int64_t u1 = u0 + (P.pre[s.i + 1] - P.pre[s.i]);
+  const int64_t u0 = static_cast<int64_t>(s.h) * P.per_head + P.pre[s.k];
+  const int64_t u1 = u0 + (P.pre[s.k + 1] - P.pre[s.k]);
   const int wa = find_worker(prm.total, W, u0);
   const int wb = find_worker(prm.total, W, u1 - 1);
   const int nslots = wb - wa + 1;
@@ -433,15 +550,23 @@ __device__ __forceinline__ void settle_partial(const DecodeKParams& prm, const S
     const int wk = wa + q;
     return (q == 0 && !a_first) ? 2 * wk + 1 : 2 * wk;
   };
-  uint16_t* obase = reinterpret_cast<uint16_t*>(prm.out) + s.i * prm.q_item_stride +
-                    (s.h * G) * kHeadDim;
-  merge_unit_warp<ACT, G>(prm.partials, obase, nslots, slot_of, lane);
+  auto out_of = [&](int r) { return row_offset<G>(prm, s, r); };
+  merge_unit_warp<ACT, R>(prm.partials, reinterpret_cast<uint16_t*>(prm.out), nslots, rows, slot_of,
+                          out_of, lane);
   // every arrival is in: re-arm the counter for the next launch (no reply needed)
   if (lane == 0) asm volatile("st.relaxed.gpu.global.s32 [%0], 0;" ::"l"(prm.counters + wa) : "memory");
 }
 
+// Query row `g` (MMA column) of a segment, or null past the unit's rows.
+template <int G, class Prm>
+__device__ __forceinline__ const uint16_t* q_row(const Prm& prm, const Seg& s, int g, int rows) {
+  if (g >= rows) return nullptr;
+  return reinterpret_cast<const uint16_t*>(prm.q) + row_offset<G>(prm, s, g);
+}
+
 // ============================================================ tensor-core path
-// Query group of G in {4, 8} query heads on the MMA N dimension (8 columns).
+// Up to 8 query rows on the MMA N dimension: a query group of G in {4, 8}
+// heads, or the side-by-side groups of a shared prefix's sibling set.
 template <int KV, int ACT, int G>
 struct MmaPath {
   static constexpr bool kF16 = (KV == kFP16) || (KV == kFP8);
@@ -450,12 +575,13 @@ struct MmaPath {
   float m0, m1, l0, l1;
   float sl2;           // logit scale in log2 units
   float vmul;          // V dequantisation scale (1 for 16-bit KV)
+  int rows;            // query rows of the segment (<= 8)
 
-  __device__ __forceinline__ void begin(const DecodeKParams& prm, const Seg& s, int lane) {
+  template <class Prm>
+  __device__ __forceinline__ void begin(const Prm& prm, const Seg& s, int lane) {
     const int g = lane >> 2, tig = lane & 3;
-    const int item = s.i;  // item index within this launch
-    const uint16_t* qrow = reinterpret_cast<const uint16_t*>(prm.q) +
-                           item * prm.q_item_stride + (s.h * G + g) * kHeadDim;
+    rows = unit_rows<G>(prm, s);
+    const uint16_t* qrow = q_row<G>(prm, s, g, rows);
     float qscale = 1.f;
     sl2 = prm.scale * kLog2e;
     vmul = 1.f;
@@ -468,7 +594,7 @@ struct MmaPath {
     }
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      if (g < G) {
+      if (qrow != nullptr) {
         if constexpr (KV == kFP8) {
           const uint2 raw = *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * tig);
           const float a = act_to_f32<ACT>(raw.x & 0xffff) * qscale;
@@ -497,7 +623,8 @@ struct MmaPath {
     else dev::mma_bf16(d, a, b0, b1);
   }
 
-  __device__ __forceinline__ void block(uint32_t ks_addr, uint32_t vs_addr, int nvalid, int lane) {
+  __device__ __forceinline__ void block(uint32_t ks_addr, uint32_t vs_addr, int nvalid, uint32_t cols,
+                                       int lane) {
     const int g = lane >> 2, tig = lane & 3;
     const int r8 = lane & 7, j = lane >> 3;
     // ---- S^T = K Q^T : 16 tokens x 8 heads
@@ -534,15 +661,22 @@ struct MmaPath {
       if (g >= nvalid) s0 = s1 = -INFINITY;
       if (g + 8 >= nvalid) s2 = s3 = -INFINITY;
     }
-    // ---- online softmax over the 16 tokens (rows) per head (column)
+    if (cols != 0xffu) {  // a sibling's own block: the other members' rows sit it out
+      if (!(cols >> (2 * tig) & 1u)) s0 = s2 = -INFINITY;
+      if (!(cols >> (2 * tig + 1) & 1u)) s1 = s3 = -INFINITY;
+    }
+    // ---- online softmax over the 16 tokens (rows) per head (column); a
+    // column that no token has reached yet keeps m = -inf and uses 0 as the
+    // reference, so its weights stay exact zeros
     const float mx0 = warp_max_rows(fmaxf(s0, s2));
     const float mx1 = warp_max_rows(fmaxf(s1, s3));
     const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float c0 = dev::exp2_approx(m0 - mn0), c1 = dev::exp2_approx(m1 - mn1);
+    const float r0 = mn0 == -INFINITY ? 0.f : mn0, r1 = mn1 == -INFINITY ? 0.f : mn1;
+    const float c0 = dev::exp2_approx(m0 - r0), c1 = dev::exp2_approx(m1 - r1);
     m0 = mn0;
     m1 = mn1;
-    const float p0 = dev::exp2_approx(s0 - mn0), p1 = dev::exp2_approx(s1 - mn1);
-    const float p2 = dev::exp2_approx(s2 - mn0), p3 = dev::exp2_approx(s3 - mn1);
+    const float p0 = dev::exp2_approx(s0 - r0), p1 = dev::exp2_approx(s1 - r1);
+    const float p2 = dev::exp2_approx(s2 - r0), p3 = dev::exp2_approx(s3 - r1);
     l0 = l0 * c0 + p0 + p2;
     l1 = l1 * c1 + p1 + p3;
     if (__any_sync(0xffffffffu, c0 != 1.f || c1 != 1.f)) {
@@ -594,21 +728,23 @@ struct MmaPath {
     else return 16 * mt + 8 * second + g;
   }
 
-  __device__ __forceinline__ void finish(const DecodeKParams& prm, const Seg& s, int lane) {
+  template <class Prm>
+  __device__ __forceinline__ void finish(const Prm& prm, const Seg& s, int lane) {
     const int g = lane >> 2, tig = lane & 3;
     const float lt0 = warp_sum_rows(l0), lt1 = warp_sum_rows(l1);
     const int h0 = 2 * tig, h1 = 2 * tig + 1;
     if (s.dest < 0) {
-      uint16_t* orow = reinterpret_cast<uint16_t*>(prm.out) + s.i * prm.q_item_stride +
-                       (s.h * G) * kHeadDim;
+      uint16_t* out = reinterpret_cast<uint16_t*>(prm.out);
+      uint16_t* orow0 = h0 < rows ? out + row_offset<G>(prm, s, h0) : nullptr;
+      uint16_t* orow1 = h1 < rows ? out + row_offset<G>(prm, s, h1) : nullptr;
       const float f0 = vmul / lt0, f1 = vmul / lt1;
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
 #pragma unroll
         for (int sec = 0; sec < 2; ++sec) {
           const int d = d_of(mt, sec, g);
-          if (h0 < G) orow[h0 * kHeadDim + d] = f32_to_act<ACT>(o[mt][2 * sec] * f0);
-          if (h1 < G) orow[h1 * kHeadDim + d] = f32_to_act<ACT>(o[mt][2 * sec + 1] * f1);
+          if (orow0) orow0[d] = f32_to_act<ACT>(o[mt][2 * sec] * f0);
+          if (orow1) orow1[d] = f32_to_act<ACT>(o[mt][2 * sec + 1] * f1);
         }
       }
     } else {
@@ -618,16 +754,22 @@ struct MmaPath {
 #pragma unroll
         for (int sec = 0; sec < 2; ++sec) {
           const int d = d_of(mt, sec, g);
-          if (h0 < G) slot[h0 * kHeadDim + d] = o[mt][2 * sec] * vmul;
-          if (h1 < G) slot[h1 * kHeadDim + d] = o[mt][2 * sec + 1] * vmul;
+          if (h0 < rows) slot[h0 * kHeadDim + d] = o[mt][2 * sec] * vmul;
+          if (h1 < rows) slot[h1 * kHeadDim + d] = o[mt][2 * sec + 1] * vmul;
         }
       }
       if (g == 0) {
         float* ml = slot + kMaxGroup * kHeadDim;
-        if (h0 < G) { ml[2 * h0] = m0; ml[2 * h0 + 1] = lt0; }
-        if (h1 < G) { ml[2 * h1] = m1; ml[2 * h1 + 1] = lt1; }
+        if (h0 < rows) { ml[2 * h0] = m0; ml[2 * h0 + 1] = lt0; }
+        if (h1 < rows) { ml[2 * h1] = m1; ml[2 * h1 + 1] = lt1; }
       }
-      settle_partial<ACT, G>(prm, s, lane);
+      if constexpr (kSibParams<Prm>) {
+        if (s.shared) {
+          settle_partial<ACT, G, kMaxGroup>(prm, s, rows, lane);
+          return;
+        }
+      }
+      settle_partial<ACT, G, G>(prm, s, G, lane);
     }
   }
 };
@@ -686,7 +828,8 @@ struct FmaPath {
     }
   }
 
-  __device__ __forceinline__ void begin(const DecodeKParams& prm, const Seg& s, int lane) {
+  template <class Prm>
+  __device__ __forceinline__ void begin(const Prm& prm, const Seg& s, int lane) {
     const int qd = lane & 3;
     sl2 = prm.scale * kLog2e;
     vmul = 1.f;
@@ -711,7 +854,9 @@ struct FmaPath {
     }
   }
 
-  __device__ __forceinline__ void block(uint32_t ks_addr, uint32_t vs_addr, int nvalid, int lane) {
+  __device__ __forceinline__ void block(uint32_t ks_addr, uint32_t vs_addr, int nvalid,
+                                       uint32_t /*cols: every row takes part in a plain unit*/,
+                                       int lane) {
     const int r = lane >> 2, qd = lane & 3;
     float s[2][G];
 #pragma unroll
@@ -785,7 +930,8 @@ struct FmaPath {
     }
   }
 
-  __device__ __forceinline__ void finish(const DecodeKParams& prm, const Seg& s, int lane) {
+  template <class Prm>
+  __device__ __forceinline__ void finish(const Prm& prm, const Seg& s, int lane) {
     const int r = lane >> 2, qd = lane & 3;
 #pragma unroll
     for (int gg = 0; gg < G; ++gg) {
@@ -833,7 +979,7 @@ struct FmaPath {
           ml[2 * gg + 1] = l[gg];
         }
       }
-      settle_partial<ACT, G>(prm, s, lane);
+      settle_partial<ACT, G, G>(prm, s, G, lane);
     }
   }
 };
@@ -842,10 +988,42 @@ template <int KV, int ACT, int G>
 using PathFor = typename std::conditional<(G >= 4), MmaPath<KV, ACT, G>, FmaPath<KV, ACT, G>>::type;
 
 // ===================================================================== kernel
-template <int KV, int ACT, int G>
+// One segment: wait for each staged block in turn, compute on it, and refill
+// the freed stage with the worker's next block.  False if a wait gave up.
+template <int KV, int G, class Path, class Prm>
+__device__ __forceinline__ bool consume_segment(Path& path, const Prm& prm, const Seg& s,
+                                                Producer<KV>& prod, const CUtensorMap* tmk,
+                                                const CUtensorMap* tmv, uint8_t* ring_ptr,
+                                                uint32_t ring, uint32_t bars, uint32_t& consumed,
+                                                int w, int lane) {
+  using T = Tile<KV>;
+  path.begin(prm, s, lane);
+#pragma unroll 1
+  for (int b = s.b0; b < s.b1; ++b) {
+    const uint32_t stage = consumed % T::kStages;
+    const uint32_t parity = (consumed / T::kStages) & 1u;
+    if (!dev::mbar_wait_bounded(bars + stage * 8, parity, kWaitLimit)) {
+      if (lane == 0) atomicOr(prm.err, kErrTimeout);
+      return false;
+    }
+    const BlockRef br = locate<G>(prm, s, b);
+    const int nvalid = max(0, min(kBlock, br.len - br.b * kBlock));
+    uint8_t* st = ring_ptr + stage * T::kStageBytes;
+    if (nvalid < kBlock) zero_tail_rows<KV>(st + T::kBytes, nvalid, lane);
+    path.block(ring + stage * T::kStageBytes, ring + stage * T::kStageBytes + T::kBytes, nvalid,
+               br.cols, lane);
+    __syncwarp();
+    ++consumed;
+    prod.issue(prm, tmk, tmv, ring, bars, w, lane);
+  }
+  path.finish(prm, s, lane);
+  return true;
+}
+
+template <int KV, int ACT, int G, class PlanT>
 __global__ void __launch_bounds__(kWarps * 32)
-    decode_kernel(const __grid_constant__ DecodeKParams prm, const __grid_constant__ CUtensorMap tmk,
-                  const __grid_constant__ CUtensorMap tmv) {
+    decode_kernel(const __grid_constant__ DecodeKParams<PlanT> prm,
+                  const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -875,36 +1053,23 @@ __global__ void __launch_bounds__(kWarps * 32)
 #pragma unroll 1
   for (int k = 0; k < T::kStages; ++k) prod.issue(prm, &tmk, &tmv, ring, bars, w, lane);
 
-  PathFor<KV, ACT, G> path;
+  // Sibling plans put every unit on the tensor cores: a set's rows fill the
+  // tile, and one path keeps the kernel within the register budget.
+  typename std::conditional<kIsSib<PlanT>, MmaPath<KV, ACT, G>, PathFor<KV, ACT, G>>::type path;
   Cursor cur;
   cur.init(prm, g0, g1, w);
   uint32_t consumed = 0;
   bool failed = false;
 #pragma unroll 1
-  while (!failed) {
+  while (true) {
     const Seg s = cur.next(prm);
     if (!s.valid) break;
-    path.begin(prm, s, lane);
-#pragma unroll 1
-    for (int b = s.b0; b < s.b1; ++b) {
-      const uint32_t stage = consumed % T::kStages;
-      const uint32_t parity = (consumed / T::kStages) & 1u;
-      if (!dev::mbar_wait_bounded(bars + stage * 8, parity, kWaitLimit)) {
-        if (lane == 0) atomicOr(prm.err, kErrTimeout);
-        failed = true;
-        break;
-      }
-      const int nvalid = min(kBlock, s.len - b * kBlock);
-      uint8_t* st = ring_ptr + stage * T::kStageBytes;
-      if (nvalid < kBlock) zero_tail_rows<KV>(st + T::kBytes, nvalid, lane);
-      path.block(ring + stage * T::kStageBytes, ring + stage * T::kStageBytes + T::kBytes, nvalid,
-                 lane);
-      __syncwarp();
-      ++consumed;
-      prod.issue(prm, &tmk, &tmv, ring, bars, w, lane);
+    const bool ok =
+        consume_segment<KV, G>(path, prm, s, prod, &tmk, &tmv, ring_ptr, ring, bars, consumed, w, lane);
+    if (!ok) {
+      failed = true;
+      break;
     }
-    if (failed) break;
-    path.finish(prm, s, lane);
   }
   if (failed) {
     // Let copies already in flight land before the CTA's shared memory goes away.
@@ -947,28 +1112,28 @@ constexpr size_t smem_bytes() {
   return 1024 + kWarps * Tile<KV>::kRingBytes + kWarps * Tile<KV>::kStages * 8;
 }
 
-template <int KV, int ACT, int G>
-cudaError_t run_decode(const DecodeKParams& prm, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                       cudaStream_t stream) {
+template <int KV, int ACT, int G, class PlanT>
+cudaError_t run_decode(const DecodeKParams<PlanT>& prm, const CUtensorMap* tmk,
+                       const CUtensorMap* tmv, cudaStream_t stream) {
   constexpr size_t smem = smem_bytes<KV>();
   static uint64_t configured = 0;  // bit per device: dynamic shared memory attribute set
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !(configured >> dev & 1u)) {
-    e = cudaFuncSetAttribute(decode_kernel<KV, ACT, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
+    e = cudaFuncSetAttribute(decode_kernel<KV, ACT, G, PlanT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     if (dev < 64) configured |= uint64_t{1} << dev;
   }
   const int grid = (prm.plan.workers + kWarps - 1) / kWarps;
-  decode_kernel<KV, ACT, G><<<grid, kWarps * 32, smem, stream>>>(prm, *tmk, *tmv);
+  decode_kernel<KV, ACT, G, PlanT><<<grid, kWarps * 32, smem, stream>>>(prm, *tmk, *tmv);
   return cudaGetLastError();
 }
 
 template <int KV, int ACT>
-cudaError_t dispatch_group(const DecodeKParams& prm, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                           cudaStream_t stream) {
+cudaError_t dispatch_group(const DecodeKParams<DecodePlan>& prm, const CUtensorMap* tmk,
+                           const CUtensorMap* tmv, cudaStream_t stream) {
   switch (prm.group) {
     case 1: return run_decode<KV, ACT, 1>(prm, tmk, tmv, stream);
     case 2: return run_decode<KV, ACT, 2>(prm, tmk, tmv, stream);
@@ -978,21 +1143,21 @@ cudaError_t dispatch_group(const DecodeKParams& prm, const CUtensorMap* tmk, con
   }
 }
 
-}  // namespace
-
-int decode_warps_per_cta() { return kWarps; }
-
-int decode_worker_capacity(int kv_dtype, int /*group*/, int num_sms) {
-  const size_t smem = kv_dtype == kFP8 ? smem_bytes<kFP8>() : smem_bytes<kBF16>();
-  const size_t per_sm = 227 * 1024;
-  const int ctas = std::max<int>(1, static_cast<int>(per_sm / smem));
-  return std::min(kMaxWorkers, num_sms * ctas * kWarps);
+// A sibling set needs members x G <= 8 rows with at least two members.
+template <int KV, int ACT>
+cudaError_t dispatch_group(const DecodeKParams<SibPlan>& prm, const CUtensorMap* tmk,
+                           const CUtensorMap* tmv, cudaStream_t stream) {
+  switch (prm.group) {
+    case 1: return run_decode<KV, ACT, 1>(prm, tmk, tmv, stream);
+    case 2: return run_decode<KV, ACT, 2>(prm, tmk, tmv, stream);
+    case 4: return run_decode<KV, ACT, 4>(prm, tmk, tmv, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
-cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                          const DecodePlan& plan, const DecodeArgs& args, cudaStream_t stream,
-                          int* launches) {
-  DecodeKParams prm;
+template <class PlanT>
+void fill_params(DecodeKParams<PlanT>& prm, const PoolView& pool, const PlanT& plan,
+                 const DecodeArgs& args) {
   prm.q = static_cast<const uint8_t*>(args.q);
   prm.out = static_cast<uint8_t*>(args.out);
   prm.tables = pool.tables;
@@ -1009,20 +1174,40 @@ cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CU
   prm.mbps = pool.mbps;
   prm.group = args.group;
   prm.total = plan.per_head * pool.num_kv_heads;
-  std::memcpy(&prm.plan, &plan, sizeof(DecodePlan));
+  std::memcpy(&prm.plan, &plan, sizeof(PlanT));
   // q / out of this launch start at item_offset
   prm.q += static_cast<int64_t>(args.item_offset) * args.q_item_stride * 2;
   prm.out += static_cast<int64_t>(args.item_offset) * args.q_item_stride * 2;
+}
 
-  cudaError_t e;
+template <class PlanT>
+cudaError_t dispatch_dtypes(const PoolView& pool, const DecodeKParams<PlanT>& prm,
+                            const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t stream) {
   if (pool.kv_dtype == kFP8) {
-    e = pool.act_dtype == kBF16 ? dispatch_group<kFP8, kBF16>(prm, tmk, tmv, stream)
-                                : dispatch_group<kFP8, kFP16>(prm, tmk, tmv, stream);
-  } else if (pool.kv_dtype == kBF16) {
-    e = dispatch_group<kBF16, kBF16>(prm, tmk, tmv, stream);
-  } else {
-    e = dispatch_group<kFP16, kFP16>(prm, tmk, tmv, stream);
+    return pool.act_dtype == kBF16 ? dispatch_group<kFP8, kBF16>(prm, tmk, tmv, stream)
+                                   : dispatch_group<kFP8, kFP16>(prm, tmk, tmv, stream);
   }
+  if (pool.kv_dtype == kBF16) return dispatch_group<kBF16, kBF16>(prm, tmk, tmv, stream);
+  return dispatch_group<kFP16, kFP16>(prm, tmk, tmv, stream);
+}
+
+}  // namespace
+
+int decode_warps_per_cta() { return kWarps; }
+
+int decode_worker_capacity(int kv_dtype, int /*group*/, int num_sms) {
+  const size_t smem = kv_dtype == kFP8 ? smem_bytes<kFP8>() : smem_bytes<kBF16>();
+  const size_t per_sm = 227 * 1024;
+  const int ctas = std::max<int>(1, static_cast<int>(per_sm / smem));
+  return std::min(kMaxWorkers, num_sms * ctas * kWarps);
+}
+
+cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                          const DecodePlan& plan, const DecodeArgs& args, cudaStream_t stream,
+                          int* launches) {
+  static thread_local DecodeKParams<DecodePlan> prm;
+  fill_params(prm, pool, plan, args);
+  cudaError_t e = dispatch_dtypes(pool, prm, tmk, tmv, stream);
   if (e != cudaSuccess) return e;
   ++*launches;
 
@@ -1040,6 +1225,16 @@ cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CU
   if (pool.act_dtype == kBF16) reduce_fixed_kernel<kBF16><<<grid, 128, 0, stream>>>(rp);
   else reduce_fixed_kernel<kFP16><<<grid, 128, 0, stream>>>(rp);
   e = cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+cudaError_t launch_decode_sib(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                              const SibPlan& plan, const DecodeArgs& args, cudaStream_t stream,
+                              int* launches) {
+  static thread_local DecodeKParams<SibPlan> prm;
+  fill_params(prm, pool, plan, args);
+  const cudaError_t e = dispatch_dtypes(pool, prm, tmk, tmv, stream);
   if (e == cudaSuccess) ++*launches;
   return e;
 }

@@ -91,6 +91,27 @@ struct DecodePlan {
   int32_t pre[kDecodeItemsCap + 1];   // prefix of per-item work units
 };
 
+// Decode work in which forks of one prompt are read together (stream-K only).
+// Sequences whose block tables start with the same run of full blocks form a
+// sibling set; the set is ONE work unit: the common prefix, read once with
+// every member's query rows side by side on the tensor-core tile (members x
+// G <= 8), followed by each member's own blocks, on which only that member's
+// rows count.  Every other sequence is a unit of its own.
+struct SibPlan {
+  int32_t n;              // items
+  int32_t nu;             // units
+  int32_t workers;
+  int32_t sets;           // units 0 .. sets-1 are sibling sets, the rest single items
+  int64_t per_head;       // KV blocks per head over all units
+  int32_t seq[kDecodeItemsCap];       // table row of each item
+  int32_t len[kDecodeItemsCap];       // tokens of each item
+  int32_t part[kDecodeItemsCap];      // first position of the item's own blocks in its unit
+  int32_t pre[kDecodeItemsCap + 1];   // prefix of per-unit block counts
+  int32_t cp[kDecodeItemsCap];        // shared full blocks at the start of the unit
+  int16_t mem0[kDecodeItemsCap + 1];  // unit u holds items mem[mem0[u] .. mem0[u+1])
+  int16_t mem[kDecodeItemsCap];
+};
+
 struct DecodeArgs {
   const void* q;
   void* out;
@@ -109,6 +130,10 @@ int decode_warps_per_cta();
 cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
                           const DecodePlan& plan, const DecodeArgs& args, cudaStream_t stream,
                           int* launches);
+// Same for a plan with shared entries; group must be 1, 2 or 4.
+cudaError_t launch_decode_sib(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                              const SibPlan& plan, const DecodeArgs& args, cudaStream_t stream,
+                              int* launches);
 
 // Thread-local text returned by pa_last_error() (defined in api.cpp).
 void set_last_error(const std::string& msg);
