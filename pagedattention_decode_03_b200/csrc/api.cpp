@@ -242,6 +242,7 @@ constexpr int kMinShareBlocks = 2;
 bool build_sib_plan(const pa_pool* p, const int32_t* seqs, int32_t cnt, int group, int cap,
                     pa::SibPlan& sp, std::vector<int32_t>& order, std::vector<int32_t>& set_of) {
   const int H = p->d.num_kv_heads;
+  const int32_t alpha = pa::stream_k_alpha(p->d.kv_dtype);
   const int max_members = pa::kMaxGroup / group;
   if (max_members < 2 || cnt < 2) return false;
   const pa::BlockManager& bm = *p->bm;
@@ -291,7 +292,7 @@ bool build_sib_plan(const pa_pool* p, const int32_t* seqs, int32_t cnt, int grou
       pos += nb_of(it) - cp;
     }
     sp.cp[nu] = cp;
-    work += pos;
+    work += alpha + pos;
     sp.pre[nu + 1] = static_cast<int32_t>(work);
     sp.mem0[nu + 1] = static_cast<int16_t>(placed);
     ++nu;
@@ -306,13 +307,15 @@ bool build_sib_plan(const pa_pool* p, const int32_t* seqs, int32_t cnt, int grou
     sp.mem[placed++] = static_cast<int16_t>(i);
     sp.part[i] = 0;
     sp.cp[nu] = 0;
-    work += nb_of(i);
+    work += alpha + nb_of(i);
     sp.pre[nu + 1] = static_cast<int32_t>(work);
     sp.mem0[nu + 1] = static_cast<int16_t>(placed);
     ++nu;
   }
   sp.n = cnt;
   sp.nu = nu;
+  sp.alpha = alpha;
+  sp.pad_ = 0;
   sp.per_head = work;
   const int64_t total = work * H;
   if (total >= (int64_t{1} << 30)) return false;
@@ -550,6 +553,7 @@ pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_
   args.scale = scale;
   args.q_item_stride = static_cast<int64_t>(num_q_heads) * pa::kHeadDim;
   static thread_local pa::DecodePlan plan;
+  const int32_t alpha = pa::stream_k_alpha(p->d.kv_dtype);
   int32_t at = 0;
   while (at < n) {
     // Items of this launch: up to the parameter capacity, and (fixed mode) the
@@ -560,7 +564,7 @@ pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_
     while (at + cnt < n && cnt < pa::kDecodeItemsCap) {
       const int32_t len = p->bm->len(seqs[at + cnt]);
       const int32_t nb = (len + 15) / 16;
-      int64_t units = nb;
+      int64_t units = nb + alpha;
       if (mode == pa::kSplitFixed) units = (nb + part_blocks - 1) / part_blocks;
       if (mode == pa::kSplitNever) units = 1;
       if (mode == pa::kSplitFixed && cnt > 0 && (work + units) * H > slots_cap) break;
@@ -577,6 +581,8 @@ pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_
     plan.n = cnt;
     plan.mode = mode;
     plan.part_blocks = part_blocks;
+    plan.alpha = mode == pa::kSplitStreamK ? alpha : 0;
+    plan.pad_ = 0;
     plan.per_head = work;
     const int64_t total = work * H;
     int64_t W = std::min<int64_t>(cap, total);
@@ -593,7 +599,7 @@ pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_
         build_sib_plan(p, seqs + at, cnt, group, cap, sib, p->order, p->set_of)) {
       e = pa::launch_decode_sib(p->view, &p->tmk, &p->tmv, sib, args, s, &launches);
       p->last_sets += sib.sets;
-      p->last_tiles += sib.per_head * H;
+      p->last_tiles += (sib.per_head - static_cast<int64_t>(sib.alpha) * sib.nu) * H;
     } else {
       e = pa::launch_decode(p->view, &p->tmk, &p->tmv, plan, args, s, &launches);
       p->last_tiles += blocks * H;

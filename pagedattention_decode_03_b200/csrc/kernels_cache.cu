@@ -28,6 +28,8 @@ struct MetaParams {
 
 template <int CAP>
 __global__ void meta_apply_kernel(const __grid_constant__ MetaParams<CAP> prm) {
+  dev::grid_dep_wait();
+  dev::grid_dep_launch();
   for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < prm.n; k += gridDim.x * blockDim.x)
     prm.meta[prm.p.v[k]] = prm.p.v[prm.n + k];
 }
@@ -48,6 +50,8 @@ struct CowParams {
 // grid.x = pairs * num_layers * 2 (K|V); each CTA copies one (layer, block) slab.
 template <int CAP>
 __global__ void __launch_bounds__(256) cow_copy_kernel(const __grid_constant__ CowParams<CAP> prm) {
+  dev::grid_dep_wait();
+  dev::grid_dep_launch();
   if (blockIdx.x == 0) {
     for (int k = threadIdx.x; k < prm.nd; k += blockDim.x)
       prm.meta[prm.p.v[2 * prm.n + k]] = prm.p.v[2 * prm.n + prm.nd + k];
@@ -83,6 +87,8 @@ struct AppendParams {
 // One warp per (token, head, K|V) row of 128 elements.
 template <int KV, int ACT, int CAP>
 __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ AppendParams<CAP> prm) {
+  dev::grid_dep_wait();
+  dev::grid_dep_launch();
   if (blockIdx.x == 0) {
     const int off = prm.T;
     for (int k = threadIdx.x; k < prm.nd; k += blockDim.x)
@@ -140,8 +146,7 @@ cudaError_t do_meta_apply(const PoolView& pool, const int32_t* idx, const int32_
   std::memcpy(prm.p.v + n, val, sizeof(int32_t) * n);
   const int threads = 256;
   const int blocks = std::max(1, std::min(64, (n + threads - 1) / threads));
-  meta_apply_kernel<CAP><<<blocks, threads, 0, stream>>>(prm);
-  return cudaGetLastError();
+  return launch_pdl(meta_apply_kernel<CAP>, dim3(blocks), dim3(threads), 0, stream, prm);
 }
 
 template <int CAP>
@@ -162,8 +167,7 @@ cudaError_t do_cow(const PoolView& pool, const int32_t* src, const int32_t* dst,
     std::memcpy(prm.p.v + 2 * n, didx, sizeof(int32_t) * nd);
     std::memcpy(prm.p.v + 2 * n + nd, dval, sizeof(int32_t) * nd);
   }
-  cow_copy_kernel<CAP><<<n * pool.num_layers * 2, 256, 0, stream>>>(prm);
-  return cudaGetLastError();
+  return launch_pdl(cow_copy_kernel<CAP>, dim3(n * pool.num_layers * 2), dim3(256), 0, stream, prm);
 }
 
 template <int KV, int ACT, int CAP>
@@ -193,8 +197,7 @@ cudaError_t do_append(const PoolView& pool, int layer, const int64_t* slots, int
   const int rows = T * pool.num_kv_heads * 2;
   const int warps = 8;
   const int blocks = std::max(1, (rows + warps - 1) / warps);
-  append_kernel<KV, ACT, CAP><<<blocks, warps * 32, 0, stream>>>(prm);
-  return cudaGetLastError();
+  return launch_pdl(append_kernel<KV, ACT, CAP>, dim3(blocks), dim3(warps * 32), 0, stream, prm);
 }
 
 template <int CAP>

@@ -107,6 +107,18 @@ __device__ __forceinline__ int find_item(const PlanT& P, int64_t r) {
   return lo;
 }
 
+// find_item, first trying `hint` and the entry after it (a worker's next
+// segment almost always starts in one of those).
+template <class PlanT>
+__device__ __forceinline__ int find_item_hint(const PlanT& P, int64_t r, int hint) {
+  const int n = n_entries(P);
+  if (hint >= 0 && hint < n && P.pre[hint] <= r) {
+    if (r < P.pre[hint + 1]) return hint;
+    if (hint + 1 < n && r < P.pre[hint + 2]) return hint + 1;
+  }
+  return find_item(P, r);
+}
+
 __device__ __forceinline__ int64_t worker_start(int64_t total, int w, int W) {
   return (total * w) / W;
 }
@@ -117,87 +129,112 @@ __device__ __forceinline__ int find_worker(int64_t total, int W, int64_t x) {
   return min(W - 1, static_cast<int>(((x + 1) * W - 1) / total));
 }
 
-// Next segment of worker `w` (whose whole share starts at g0) within the
-// remaining range [g, g_end).
+// Stream-K piece of one unit.  A unit occupies alpha + nb positions of the
+// work axis: alpha positions that stand for the fixed cost of a segment
+// (begin, finish, partial write and arrival) and carry no block, then its nb
+// KV blocks.  Shares are equal in positions, so a worker whose share crosses
+// unit boundaries gets fewer blocks.  From position r (offset o = r - v0 in
+// the unit [v0, v1)) the worker takes `take` positions; the piece reads blocks
+// [b0, b1).  Returns false when those positions hold no block.  A piece that
+// covers the unit's blocks only in part writes partial slot 2w if it starts
+// inside the blocks (it holds the share's start; one per worker), else 2w+1
+// (it holds the share's end).
+__device__ __forceinline__ bool stream_piece(int64_t r, int32_t v0, int32_t v1, int32_t alpha,
+                                             int64_t avail, int w, int64_t& take, Seg& s) {
+  const int32_t unit_nb = v1 - v0 - alpha;
+  take = min(static_cast<int64_t>(v1) - r, avail);
+  const int64_t o = r - v0;
+  s.b0 = static_cast<int32_t>(max(o - alpha, int64_t{0}));
+  s.b1 = static_cast<int32_t>(max(o + take - alpha, int64_t{0}));
+  if (s.b1 <= s.b0) return false;
+  const bool whole = s.b0 == 0 && s.b1 == unit_nb;
+  s.dest = whole ? -1 : (s.b0 > 0 ? 2 * w : 2 * w + 1);
+  return true;
+}
+
+// Next segment of worker `w` within the remaining range [g, g_end) of its
+// share; `hint` carries the entry of the previous segment.
 __device__ __forceinline__ Seg next_seg(const DecodeKParams<DecodePlan>& prm, int64_t& g,
-                                        int64_t g_end, int w, int64_t g0) {
+                                        int64_t g_end, int w, int64_t /*g0*/, int& hint) {
   Seg s;
-  s.valid = g < g_end;
   s.shared = false;
-  if (!s.valid) return s;
   const DecodePlan& P = prm.plan;
   const int64_t per_head = P.per_head;
-  s.h = static_cast<int32_t>(g / per_head);
-  const int64_t r = g - static_cast<int64_t>(s.h) * per_head;
-  if (P.mode == kSplitNever) {
-    s.i = static_cast<int32_t>(r);
-  } else {
-    s.i = find_item(P, r);
-  }
-  s.k = s.i;
-  s.seq = P.seq[s.i];
-  s.len = P.len[s.i];
-  int32_t nb = (s.len + kBlock - 1) / kBlock;
-  if (s.len <= 0 || nb > prm.mbps) {
-    atomicOr(prm.err, kErrBadLen);
-    nb = min(max(nb, 1), prm.mbps);
-    s.len = max(s.len, 1);
-  }
-  if (P.mode == kSplitStreamK) {
-    const int32_t unit_nb = P.pre[s.i + 1] - P.pre[s.i];
-    if (unit_nb != nb) atomicOr(prm.err, kErrBadLen);
-    s.b0 = static_cast<int32_t>(r - P.pre[s.i]);
-    const int64_t take = min(static_cast<int64_t>(unit_nb - s.b0), g_end - g);
-    s.b1 = s.b0 + static_cast<int32_t>(take);
-    const bool whole = s.b0 == 0 && s.b1 == unit_nb;
-    s.dest = whole ? -1 : (g == g0 ? 2 * w : 2 * w + 1);
-    g += take;
-  } else if (P.mode == kSplitFixed) {
-    const int32_t p = static_cast<int32_t>(r - P.pre[s.i]);
-    const int32_t np = P.pre[s.i + 1] - P.pre[s.i];
-    s.b0 = p * P.part_blocks;
-    s.b1 = min(nb, s.b0 + P.part_blocks);
-    if (s.b0 >= s.b1) {  // inconsistent lengths: clamp to an empty-free range
-      atomicOr(prm.err, kErrBadLen);
-      s.b0 = max(0, s.b1 - 1);
+  for (;;) {
+    s.valid = g < g_end;
+    if (!s.valid) return s;
+    s.h = static_cast<int32_t>(g / per_head);
+    const int64_t r = g - static_cast<int64_t>(s.h) * per_head;
+    if (P.mode == kSplitNever) {
+      s.i = static_cast<int32_t>(r);
+    } else {
+      s.i = find_item_hint(P, r, hint);
+      hint = s.i;
     }
-    s.dest = np == 1 ? -1 : static_cast<int32_t>(g);
-    g += 1;
-  } else {
-    s.b0 = 0;
-    s.b1 = nb;
-    s.dest = -1;
-    g += 1;
+    s.k = s.i;
+    s.seq = P.seq[s.i];
+    s.len = P.len[s.i];
+    int32_t nb = (s.len + kBlock - 1) / kBlock;
+    if (s.len <= 0 || nb > prm.mbps) {
+      atomicOr(prm.err, kErrBadLen);
+      nb = min(max(nb, 1), prm.mbps);
+      s.len = max(s.len, 1);
+    }
+    if (P.mode == kSplitStreamK) {
+      const int32_t v0 = P.pre[s.i], v1 = P.pre[s.i + 1];
+      if (v1 - v0 - P.alpha != nb) atomicOr(prm.err, kErrBadLen);
+      int64_t take;
+      const bool any = stream_piece(r, v0, v1, P.alpha, g_end - g, w, take, s);
+      g += take;
+      if (!any) continue;
+    } else if (P.mode == kSplitFixed) {
+      const int32_t p = static_cast<int32_t>(r - P.pre[s.i]);
+      const int32_t np = P.pre[s.i + 1] - P.pre[s.i];
+      s.b0 = p * P.part_blocks;
+      s.b1 = min(nb, s.b0 + P.part_blocks);
+      if (s.b0 >= s.b1) {  // inconsistent lengths: clamp to an empty-free range
+        atomicOr(prm.err, kErrBadLen);
+        s.b0 = max(0, s.b1 - 1);
+      }
+      s.dest = np == 1 ? -1 : static_cast<int32_t>(g);
+      g += 1;
+    } else {
+      s.b0 = 0;
+      s.b1 = nb;
+      s.dest = -1;
+      g += 1;
+    }
+    return s;
   }
-  return s;
 }
 
 // Sibling plan (always stream-K): same cutting and partial slots as a plain
 // stream-K plan, over units that may hold several items.
 __device__ __forceinline__ Seg next_seg(const DecodeKParams<SibPlan>& prm, int64_t& g,
-                                        int64_t g_end, int w, int64_t g0) {
+                                        int64_t g_end, int w, int64_t /*g0*/, int& hint) {
   Seg s;
-  s.valid = g < g_end;
-  if (!s.valid) return s;
   const SibPlan& P = prm.plan;
-  s.h = static_cast<int32_t>(g / P.per_head);
-  const int64_t r = g - static_cast<int64_t>(s.h) * P.per_head;
-  s.k = find_item(P, r);
-  const int m0 = P.mem0[s.k];
-  s.shared = P.mem0[s.k + 1] - m0 > 1;
-  s.i = P.mem[m0];
-  s.seq = P.seq[s.i];
-  s.len = P.len[s.i];
-  const int32_t unit_nb = P.pre[s.k + 1] - P.pre[s.k];
-  if (!s.shared && (s.len <= 0 || (s.len + kBlock - 1) / kBlock != unit_nb || unit_nb > prm.mbps))
-    atomicOr(prm.err, kErrBadLen);
-  s.b0 = static_cast<int32_t>(r - P.pre[s.k]);
-  const int64_t take = min(static_cast<int64_t>(unit_nb - s.b0), g_end - g);
-  s.b1 = s.b0 + static_cast<int32_t>(take);
-  const bool whole = s.b0 == 0 && s.b1 == unit_nb;
-  s.dest = whole ? -1 : (g == g0 ? 2 * w : 2 * w + 1);
-  g += take;
-  return s;
+  for (;;) {
+    s.valid = g < g_end;
+    if (!s.valid) return s;
+    s.h = static_cast<int32_t>(g / P.per_head);
+    const int64_t r = g - static_cast<int64_t>(s.h) * P.per_head;
+    s.k = find_item_hint(P, r, hint);
+    hint = s.k;
+    const int m0 = P.mem0[s.k];
+    s.shared = P.mem0[s.k + 1] - m0 > 1;
+    s.i = P.mem[m0];
+    s.seq = P.seq[s.i];
+    s.len = P.len[s.i];
+    const int32_t v0 = P.pre[s.k], v1 = P.pre[s.k + 1];
+    const int32_t unit_nb = v1 - v0 - P.alpha;
+    if (!s.shared && (s.len <= 0 || (s.len + kBlock - 1) / kBlock != unit_nb || unit_nb > prm.mbps))
+      atomicOr(prm.err, kErrBadLen);
+    int64_t take;
+    const bool any = stream_piece(r, v0, v1, P.alpha, g_end - g, w, take, s);
+    g += take;
+    if (any) return s;
+  }
 }
 
 // Where position o of segment s lives.  Plain plans: block o of the item.
@@ -234,6 +271,7 @@ __device__ __forceinline__ BlockRef locate(const DecodeKParams<SibPlan>& prm, co
 struct Cursor {
   int64_t g, end, g0, glast;
   int w;
+  int hint, hint_g0;  // entry of the next segment, and of the share's start
   bool second;
 
   template <class Prm>
@@ -241,12 +279,29 @@ struct Cursor {
     g0 = s0;
     w = wk;
     glast = s0;
+    hint = hint_g0 = -1;
     const auto& P = prm.plan;
     if (plan_mode(P) == kSplitStreamK && s1 > s0) {
+      // entries of the share's last and first positions, two searches
+      // interleaved so their dependent loads overlap
       const int64_t x = s1 - 1;
       const int64_t h = x / P.per_head;
-      const int i = find_item(P, x - h * P.per_head);
-      glast = max(s0, h * P.per_head + P.pre[i]);
+      const int64_t r1 = x - h * P.per_head;
+      const int64_t r0 = s0 - (s0 / P.per_head) * P.per_head;
+      int lo1 = 0, hi1 = n_entries(P) - 1, lo0 = 0, hi0 = hi1;
+      while (lo1 < hi1 || lo0 < hi0) {
+        if (lo1 < hi1) {
+          const int mid = (lo1 + hi1 + 1) >> 1;
+          if (P.pre[mid] <= r1) lo1 = mid; else hi1 = mid - 1;
+        }
+        if (lo0 < hi0) {
+          const int mid = (lo0 + hi0 + 1) >> 1;
+          if (P.pre[mid] <= r0) lo0 = mid; else hi0 = mid - 1;
+        }
+      }
+      glast = max(s0, h * P.per_head + P.pre[lo1]);
+      hint = lo1;
+      hint_g0 = lo0;
     }
     g = glast;
     end = s1;
@@ -255,12 +310,17 @@ struct Cursor {
 
   template <class Prm>
   __device__ __forceinline__ Seg next(const Prm& prm) {
-    if (g >= end && !second && glast > g0) {
-      second = true;
-      g = g0;
-      end = glast;
+    for (;;) {
+      if (g >= end && !second && glast > g0) {
+        second = true;
+        g = g0;
+        end = glast;
+        hint = hint_g0;
+      }
+      const Seg s = next_seg(prm, g, end, w, g0, hint);
+      // the first phase may hold only cost positions: go on with the second
+      if (s.valid || second || glast <= g0) return s;
     }
-    return next_seg(prm, g, end, w, g0);
   }
 };
 
@@ -270,15 +330,16 @@ struct Producer {
   Cursor cur;
   Seg seg;
   int32_t b;          // next block of seg to fetch
-  int32_t tc_val, tc_base, tc_seq;
+  int32_t tc_val, tc_base, tc_unit;
   uint32_t issued;
 
+  // Starts from a copy of the consumer's cursor (same segments, same order).
   template <class Prm>
-  __device__ __forceinline__ void init(const Prm& prm, int64_t g0, int64_t g1, int w) {
-    cur.init(prm, g0, g1, w);
+  __device__ __forceinline__ void init(const Prm& prm, const Cursor& c) {
+    cur = c;
     seg = cur.next(prm);
     b = seg.b0;
-    tc_seq = -1;
+    tc_unit = -1;
     tc_base = 0;
     tc_val = 0;
     issued = 0;
@@ -295,14 +356,15 @@ struct Producer {
       if (!seg.valid) return;
       b = seg.b0;
     }
-    const BlockRef br = locate<1>(prm, seg, b);
-    if (br.seq != tc_seq || br.b < tc_base || br.b >= tc_base + 32) {
-      tc_seq = br.seq;
-      tc_base = br.b;
-      const int idx = br.b + lane;
-      tc_val = idx >= 0 && idx < prm.mbps ? prm.tables[static_cast<int64_t>(br.seq) * prm.mbps + idx] : 0;
+    // physical ids of the unit's positions b .. b+31, one per lane (a sibling
+    // set's positions run through several table rows)
+    if (seg.k != tc_unit || b < tc_base || b >= tc_base + 32) {
+      tc_unit = seg.k;
+      tc_base = b;
+      const BlockRef r = locate<1>(prm, seg, b + lane);
+      tc_val = r.b >= 0 && r.b < prm.mbps ? prm.tables[static_cast<int64_t>(r.seq) * prm.mbps + r.b] : 0;
     }
-    int32_t phys = __shfl_sync(0xffffffffu, tc_val, br.b - tc_base);
+    int32_t phys = __shfl_sync(0xffffffffu, tc_val, b - tc_base);
     if (static_cast<uint32_t>(phys) >= static_cast<uint32_t>(prm.num_blocks)) {
       if (lane == 0) atomicOr(prm.err, kErrBadBlock);
       phys = 0;
@@ -532,8 +594,9 @@ __device__ __forceinline__ void settle_partial(const Prm& prm, const Seg& s, int
   const auto& P = prm.plan;
   if (plan_mode(P) != kSplitStreamK) return;  // fixed partitions: a separate reduce kernel merges
   const int W = P.workers;
-  const int64_t u0 = static_cast<int64_t>(s.h) * P.per_head + P.pre[s.k];
-  const int64_t u1 = u0 + (P.pre[s.k + 1] - P.pre[s.k]);
+  // the unit's blocks: positions [u0, u1) (after its alpha cost positions)
+  const int64_t u0 = static_cast<int64_t>(s.h) * P.per_head + P.pre[s.k] + P.alpha;
+  const int64_t u1 = static_cast<int64_t>(s.h) * P.per_head + P.pre[s.k + 1];
   const int wa = find_worker(prm.total, W, u0);
   const int wb = find_worker(prm.total, W, u1 - 1);
   const int nslots = wb - wa + 1;
@@ -545,10 +608,11 @@ __device__ __forceinline__ void settle_partial(const Prm& prm, const Seg& s, int
   old = __shfl_sync(0xffffffffu, old, 0);
   if (old != nslots - 1) return;
   __syncwarp();
-  const bool a_first = worker_start(prm.total, wa, W) == u0;
+  // wa's piece starts inside the blocks (slot 2wa) only if its share does
+  const bool a_inside = worker_start(prm.total, wa, W) > u0;
   auto slot_of = [&](int q) {
     const int wk = wa + q;
-    return (q == 0 && !a_first) ? 2 * wk + 1 : 2 * wk;
+    return (q == 0 && !a_inside) ? 2 * wk + 1 : 2 * wk;
   };
   auto out_of = [&](int r) { return row_offset<G>(prm, s, r); };
   merge_unit_warp<ACT, R>(prm.partials, reinterpret_cast<uint16_t*>(prm.out), nslots, rows, slot_of,
@@ -1049,15 +1113,17 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int64_t g0 = worker_start(prm.total, w, W);
   const int64_t g1 = worker_start(prm.total, w + 1, W);
   Producer<KV> prod;
-  prod.init(prm, g0, g1, w);
+  Cursor cur;
+  cur.init(prm, g0, g1, w);  // kernel parameters only: may overlap the previous kernel
+  dev::grid_dep_wait();
+  dev::grid_dep_launch();
+  prod.init(prm, cur);
 #pragma unroll 1
   for (int k = 0; k < T::kStages; ++k) prod.issue(prm, &tmk, &tmv, ring, bars, w, lane);
 
   // Sibling plans put every unit on the tensor cores: a set's rows fill the
   // tile, and one path keeps the kernel within the register budget.
   typename std::conditional<kIsSib<PlanT>, MmaPath<KV, ACT, G>, PathFor<KV, ACT, G>>::type path;
-  Cursor cur;
-  cur.init(prm, g0, g1, w);
   uint32_t consumed = 0;
   bool failed = false;
 #pragma unroll 1
@@ -1092,6 +1158,8 @@ struct ReduceKParams {
 // item's partitions (if there is more than one) into the output.
 template <int ACT>
 __global__ void __launch_bounds__(128) reduce_fixed_kernel(const __grid_constant__ ReduceKParams prm) {
+  dev::grid_dep_wait();
+  dev::grid_dep_launch();
   const DecodePlan& P = prm.plan;
   const int h = blockIdx.x / P.n;
   const int i = blockIdx.x - h * P.n;
@@ -1127,8 +1195,8 @@ cudaError_t run_decode(const DecodeKParams<PlanT>& prm, const CUtensorMap* tmk,
     if (dev < 64) configured |= uint64_t{1} << dev;
   }
   const int grid = (prm.plan.workers + kWarps - 1) / kWarps;
-  decode_kernel<KV, ACT, G, PlanT><<<grid, kWarps * 32, smem, stream>>>(prm, *tmk, *tmv);
-  return cudaGetLastError();
+  return launch_pdl(decode_kernel<KV, ACT, G, PlanT>, dim3(grid), dim3(kWarps * 32), smem, stream,
+                    prm, *tmk, *tmv);
 }
 
 template <int KV, int ACT>
@@ -1222,9 +1290,9 @@ cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CU
   rp.total = prm.total;
   std::memcpy(&rp.plan, &plan, sizeof(DecodePlan));
   const int grid = plan.n * pool.num_kv_heads;
-  if (pool.act_dtype == kBF16) reduce_fixed_kernel<kBF16><<<grid, 128, 0, stream>>>(rp);
-  else reduce_fixed_kernel<kFP16><<<grid, 128, 0, stream>>>(rp);
-  e = cudaGetLastError();
+  e = pool.act_dtype == kBF16
+          ? launch_pdl(reduce_fixed_kernel<kBF16>, dim3(grid), dim3(128), 0, stream, rp)
+          : launch_pdl(reduce_fixed_kernel<kFP16>, dim3(grid), dim3(128), 0, stream, rp);
   if (e == cudaSuccess) ++*launches;
   return e;
 }

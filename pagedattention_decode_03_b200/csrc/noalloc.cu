@@ -132,6 +132,7 @@ extern "C" pa_status pa_decode_attention_noalloc(const pa_pool_desc* d, int32_t 
     return fail(PA_ERR_INVALID_ARG, "block tables too large");
   static thread_local pa::DecodePlan plan;
   int64_t work = 0;
+  const int32_t alpha = pa::stream_k_alpha(d->kv_dtype);
   plan.pre[0] = 0;
   for (int32_t i = 0; i < n; ++i) {
     const int32_t len = seq_lens[i];
@@ -140,7 +141,7 @@ extern "C" pa_status pa_decode_attention_noalloc(const pa_pool_desc* d, int32_t 
                                           ": length must be in [1, max_blocks_per_seq * 16]");
     plan.seq[i] = i;  // row i of the caller's block tables
     plan.len[i] = len;
-    work += (len + 15) / 16;
+    work += alpha + (len + 15) / 16;
     plan.pre[i + 1] = static_cast<int32_t>(work);
   }
   if (work * d->num_kv_heads >= (int64_t{1} << 30))
@@ -215,6 +216,8 @@ extern "C" pa_status pa_decode_attention_noalloc(const pa_pool_desc* d, int32_t 
   plan.n = n;
   plan.mode = pa::kSplitStreamK;
   plan.part_blocks = 0;
+  plan.alpha = alpha;
+  plan.pad_ = 0;
   plan.per_head = work;
   plan.workers = static_cast<int32_t>(std::max<int64_t>(1, W));
   pa::DecodeArgs args;

@@ -85,7 +85,9 @@ struct DecodePlan {
   int32_t mode;           // SplitMode
   int32_t part_blocks;    // fixed mode: blocks per partition
   int32_t workers;        // warps that carry work
-  int64_t per_head;       // work units per KV head (Tn / Pn / n)
+  int32_t alpha;          // stream-K: cost positions in front of each item's blocks
+  int32_t pad_;
+  int64_t per_head;       // work positions per KV head (stream-K: sum of alpha + blocks)
   int32_t seq[kDecodeItemsCap];       // table row of each item
   int32_t len[kDecodeItemsCap];       // tokens of each item
   int32_t pre[kDecodeItemsCap + 1];   // prefix of per-item work units
@@ -102,7 +104,9 @@ struct SibPlan {
   int32_t nu;             // units
   int32_t workers;
   int32_t sets;           // units 0 .. sets-1 are sibling sets, the rest single items
-  int64_t per_head;       // KV blocks per head over all units
+  int32_t alpha;          // cost positions in front of each unit's blocks
+  int32_t pad_;
+  int64_t per_head;       // work positions per head: sum over units of alpha + blocks
   int32_t seq[kDecodeItemsCap];       // table row of each item
   int32_t len[kDecodeItemsCap];       // tokens of each item
   int32_t part[kDecodeItemsCap];      // first position of the item's own blocks in its unit
@@ -122,6 +126,14 @@ struct DecodeArgs {
   int64_t q_item_stride;  // elements between consecutive items of q / out (num_q_heads*128)
   int32_t item_offset;    // index of plan item 0 within the caller's arrays
 };
+
+// Stream-K cost positions per work unit, in KV blocks: they stand for the
+// fixed cost of a segment (query load, finish, partial write, arrival, the
+// merge) and, by shrinking the shares of workers that cross unit boundaries,
+// also move boundaries off units so fewer units are cut.  Chosen by a sweep
+// on B200 (0 .. 16 for 16-bit and FP8 KV; 8B-, 70B- and 7B-class layers and
+// 32K-token FP8): 12 was best or within noise of best everywhere.
+inline int32_t stream_k_alpha(int32_t /*kv_dtype*/) { return 12; }
 
 // Number of decode workers (warps) that fit on the device at once.
 int decode_worker_capacity(int kv_dtype, int group, int num_sms);
