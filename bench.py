@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--layers", type=int, default=None,
+                    help="profiling: keep only the first N layers (a smaller case of the same "
+                         "kernels; the JSON line then names the reduced workload)")
     return ap.parse_args()
 
 
@@ -68,6 +71,15 @@ def pool_steps(a):
     """Decode steps the pool is sized for (same in both arms): the timed run
     plus the end-to-end run, and never fewer than the workload's own count."""
     return max(DEFAULT_STEPS[a.workload], 2 * (a.warmup + a.steps))
+
+
+def make_workload(a, seed):
+    import dataclasses
+    import workloads
+    w = workloads.workload(a.workload, seed=seed, steps=pool_steps(a))
+    if a.layers:
+        w = dataclasses.replace(w, num_layers=max(1, min(a.layers, w.num_layers)))
+    return w
 
 
 def peaks():
@@ -336,7 +348,7 @@ def run_ours(a, rank, world, local_rank):
         _b.build()
     if world > 1:
         torch.distributed.barrier()
-    w = workloads.workload(a.workload, seed=a.seed + rank, steps=pool_steps(a))
+    w = make_workload(a, a.seed + rank)
     partition = w.partition_tokens if a.partition is None else a.partition
     r = Runner(w, device, partition, a.seed + rank)
     stream_obj = torch.cuda.current_stream(device)
@@ -546,7 +558,7 @@ def _subset(w, seqs):
 
 def run_reference(a):
     import workloads
-    w = workloads.workload(a.workload, seed=a.seed, steps=pool_steps(a))
+    w = make_workload(a, a.seed)
     partition = w.partition_tokens if a.partition is None else a.partition
     lens0 = w.lens_before_step(0)
     smp = OracleSample(w, lens0)

@@ -586,7 +586,12 @@ pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_
     plan.per_head = work;
     const int64_t total = work * H;
     int64_t W = std::min<int64_t>(cap, total);
-    if (mode == pa::kSplitStreamK) {
+    if (mode != pa::kSplitStreamK) {
+      // whole partitions (or sequences) per worker: the same count for every
+      // worker, so no worker runs a round more than the others
+      const int64_t rounds = (total + cap - 1) / cap;
+      W = (total + rounds - 1) / rounds;
+    } else {
       W = std::min<int64_t>(W, std::max<int64_t>(1, (total + kMinBlocksPerWorker - 1) / kMinBlocksPerWorker));
       W = std::min<int64_t>(W, slots_cap / 2);
     }

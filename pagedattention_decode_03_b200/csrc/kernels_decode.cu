@@ -440,7 +440,10 @@ __device__ __forceinline__ uint16_t f32_to_act(float x) {
 // ================================================================ LSE merge
 // One warp merges query row `gg` over `nslots` partial slots (m, l, o~):
 //   M = max m_k,  L = sum 2^(m_k - M) l_k,  out = sum 2^(m_k - M) o~_k / L.
-// Partials written by other SMs are read through L2 (ld.global.cg).
+// Partials written by other SMs are read through L2 (ld.global.cg).  The
+// (m, l) pairs are read 32 slots at a time across the lanes; the o~ rows
+// kInFlight slots at a time, every load of a batch issued before any use, so
+// a row of many partitions costs nslots / kInFlight round trips, not nslots.
 template <int ACT, class SlotFn>
 __device__ __forceinline__ void merge_row(const float* partials, uint16_t* orow, int gg, int nslots,
                                           SlotFn slot_of, int lane) {
@@ -452,25 +455,37 @@ __device__ __forceinline__ void merge_row(const float* partials, uint16_t* orow,
   for (int k = lane; k < nslots; k += 32) M = fmaxf(M, __ldcg(ml_of(k)));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  constexpr int kInFlight = 32;  // one batch per 32 slots
   float L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int k0 = 0; k0 < nslots; k0 += 32) {
     const int k = k0 + lane;
     float wk = 0.f;
     if (k < nslots) {
-      const float* ml = ml_of(k);
-      wk = dev::exp2_approx(__ldcg(ml) - M);
-      L += wk * __ldcg(ml + 1);
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(ml_of(k)));
+      wk = dev::exp2_approx(ml.x - M);
+      L += wk * ml.y;
     }
     const int cnt = min(32, nslots - k0);
-    for (int j = 0; j < cnt; ++j) {
-      const float wj = __shfl_sync(0xffffffffu, wk, j);
-      const float4 x = __ldcg(reinterpret_cast<const float4*>(
-          partials + static_cast<int64_t>(slot_of(k0 + j)) * kPartialSlotFloats + gg * kHeadDim) + lane);
-      acc.x += wj * x.x;
-      acc.y += wj * x.y;
-      acc.z += wj * x.z;
-      acc.w += wj * x.w;
+    for (int j0 = 0; j0 < cnt; j0 += kInFlight) {
+      float4 x[kInFlight];
+#pragma unroll
+      for (int t = 0; t < kInFlight; ++t) {
+        if (j0 + t < cnt)
+          x[t] = __ldcg(reinterpret_cast<const float4*>(
+                            partials + static_cast<int64_t>(slot_of(k0 + j0 + t)) * kPartialSlotFloats +
+                            gg * kHeadDim) + lane);
+      }
+#pragma unroll
+      for (int t = 0; t < kInFlight; ++t) {
+        const float wj = __shfl_sync(0xffffffffu, wk, (j0 + t) & 31);
+        if (j0 + t < cnt) {
+          acc.x += wj * x[t].x;
+          acc.y += wj * x[t].y;
+          acc.z += wj * x[t].z;
+          acc.w += wj * x[t].w;
+        }
+      }
     }
   }
 #pragma unroll
@@ -1154,10 +1169,11 @@ struct ReduceKParams {
   DecodePlan plan;
 };
 
-// Fixed partitions: CTA = (head, item); each warp merges query rows of the
-// item's partitions (if there is more than one) into the output.
+// Fixed partitions: CTA = (head, item), one warp per query row of the group;
+// each merges that row over the item's partitions (if there is more than one)
+// into the output.
 template <int ACT>
-__global__ void __launch_bounds__(128) reduce_fixed_kernel(const __grid_constant__ ReduceKParams prm) {
+__global__ void __launch_bounds__(kMaxGroup * 32) reduce_fixed_kernel(const __grid_constant__ ReduceKParams prm) {
   dev::grid_dep_wait();
   dev::grid_dep_launch();
   const DecodePlan& P = prm.plan;
@@ -1291,8 +1307,8 @@ cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CU
   std::memcpy(&rp.plan, &plan, sizeof(DecodePlan));
   const int grid = plan.n * pool.num_kv_heads;
   e = pool.act_dtype == kBF16
-          ? launch_pdl(reduce_fixed_kernel<kBF16>, dim3(grid), dim3(128), 0, stream, rp)
-          : launch_pdl(reduce_fixed_kernel<kFP16>, dim3(grid), dim3(128), 0, stream, rp);
+          ? launch_pdl(reduce_fixed_kernel<kBF16>, dim3(grid), dim3(32 * args.group), 0, stream, rp)
+          : launch_pdl(reduce_fixed_kernel<kFP16>, dim3(grid), dim3(32 * args.group), 0, stream, rp);
   if (e == cudaSuccess) ++*launches;
   return e;
 }
