@@ -476,9 +476,44 @@ def run_ours(a, rank, world, local_rank):
         "clocks": clk.summary(),
         "e2e": e2e,
     }
+    if w.name == "tiny":
+        line["graph_batch"] = graph_batch(r, 1000)
     if rank == 0 and not a.no_cpu:
         line["cpu_baseline"] = cpu_baseline(w, a.cpu_seconds, lens0)
     return line
+
+
+def graph_batch(r, reps):
+    """GPU time of one decode launch of a launch-bound workload: `reps` decodes of
+    layer 0 (same lengths, no appends) captured in one CUDA graph and replayed
+    once.  L2-warm (the tiny KV pool stays in L2), so it shows the launch and
+    ramp cost, not HBM bandwidth."""
+    import torch
+    w, L = r.w, r.L
+    n = len(r.seqs)
+    sp = r.seqs.ctypes.data_as(r.i32p)
+    q, out = ctypes.c_void_p(r.q[0][0].data_ptr()), ctypes.c_void_p(r.out[0].data_ptr())
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        cs = ctypes.c_void_p(side.cuda_stream)
+        for _ in range(reps):
+            st = L.pa_decode_attention(r.pool.handle, 0, n, sp, w.num_q_heads, q, out,
+                                       ctypes.c_float(w.scale), r.partition, cs)
+            if st != 0:
+                raise RuntimeError(f"pa_decode_attention (graph capture): {r.pa.pa_last_error()}")
+    torch.cuda.synchronize()
+    g.replay()                      # warm-up replay
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return {"launches": reps, "us_per_decode": round(e0.elapsed_time(e1) * 1e3 / reps, 2),
+            "note": "L2-warm: one decode of layer 0 replayed from a CUDA graph"}
 
 
 # ==================================================================== oracle
