@@ -438,64 +438,58 @@ __device__ __forceinline__ uint16_t f32_to_act(float x) {
 }
 
 // ================================================================ LSE merge
-// One warp merges query row `gg` over `nslots` partial slots (m, l, o~):
-//   M = max m_k,  L = sum 2^(m_k - M) l_k,  out = sum 2^(m_k - M) o~_k / L.
-// Partials written by other SMs are read through L2 (ld.global.cg).  The
-// (m, l) pairs are read 32 slots at a time across the lanes; the o~ rows
-// kInFlight slots at a time, every load of a batch issued before any use, so
-// a row of many partitions costs nslots / kInFlight round trips, not nslots.
-template <int ACT, class SlotFn>
-__device__ __forceinline__ void merge_row(const float* partials, uint16_t* orow, int gg, int nslots,
-                                          SlotFn slot_of, int lane) {
+// One warp's share of a log-sum-exp merge: query row `gg` over partial slots
+// kb .. ke-1, each (m, l, o~).  Leaves M = max m_k, L = sum 2^(m_k - M) l_k and
+// acc = sum 2^(m_k - M) o~_k (d = 4*lane .. 4*lane+3), unnormalised; M = -inf
+// for an empty range.  Partials written by other SMs are read through L2
+// (ld.global.cg): the (m, l) pairs 32 slots at a time across the lanes, the o~
+// rows 32 slots at a time with every load issued before any use.
+template <class SlotFn>
+__device__ __forceinline__ void merge_row_part(const float* partials, int gg, int kb, int ke,
+                                               SlotFn slot_of, int lane, float& M, float& L,
+                                               float4& acc) {
   auto ml_of = [&](int k) {
     return partials + static_cast<int64_t>(slot_of(k)) * kPartialSlotFloats + kMaxGroup * kHeadDim +
            2 * gg;
   };
-  float M = -INFINITY;
-  for (int k = lane; k < nslots; k += 32) M = fmaxf(M, __ldcg(ml_of(k)));
+  M = -INFINITY;
+  for (int k = kb + lane; k < ke; k += 32) M = fmaxf(M, __ldcg(ml_of(k)));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  constexpr int kInFlight = 32;  // one batch per 32 slots
-  float L = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int k0 = 0; k0 < nslots; k0 += 32) {
+  const float ref = M == -INFINITY ? 0.f : M;
+  constexpr int kInFlight = 32;
+  L = 0.f;
+  acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k0 = kb; k0 < ke; k0 += kInFlight) {
     const int k = k0 + lane;
     float wk = 0.f;
-    if (k < nslots) {
+    if (k < ke) {
       const float2 ml = __ldcg(reinterpret_cast<const float2*>(ml_of(k)));
-      wk = dev::exp2_approx(ml.x - M);
+      wk = dev::exp2_approx(ml.x - ref);
       L += wk * ml.y;
     }
-    const int cnt = min(32, nslots - k0);
-    for (int j0 = 0; j0 < cnt; j0 += kInFlight) {
-      float4 x[kInFlight];
+    const int cnt = min(kInFlight, ke - k0);
+    float4 x[kInFlight];
 #pragma unroll
-      for (int t = 0; t < kInFlight; ++t) {
-        if (j0 + t < cnt)
-          x[t] = __ldcg(reinterpret_cast<const float4*>(
-                            partials + static_cast<int64_t>(slot_of(k0 + j0 + t)) * kPartialSlotFloats +
-                            gg * kHeadDim) + lane);
-      }
+    for (int t = 0; t < kInFlight; ++t) {
+      if (t < cnt)
+        x[t] = __ldcg(reinterpret_cast<const float4*>(
+                          partials + static_cast<int64_t>(slot_of(k0 + t)) * kPartialSlotFloats +
+                          gg * kHeadDim) + lane);
+    }
 #pragma unroll
-      for (int t = 0; t < kInFlight; ++t) {
-        const float wj = __shfl_sync(0xffffffffu, wk, (j0 + t) & 31);
-        if (j0 + t < cnt) {
-          acc.x += wj * x[t].x;
-          acc.y += wj * x[t].y;
-          acc.z += wj * x[t].z;
-          acc.w += wj * x[t].w;
-        }
+    for (int t = 0; t < kInFlight; ++t) {
+      const float wj = __shfl_sync(0xffffffffu, wk, t);
+      if (t < cnt) {
+        acc.x += wj * x[t].x;
+        acc.y += wj * x[t].y;
+        acc.z += wj * x[t].z;
+        acc.w += wj * x[t].w;
       }
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  const float inv = 1.f / L;
-  const uint32_t a = static_cast<uint32_t>(f32_to_act<ACT>(acc.x * inv)) |
-                     (static_cast<uint32_t>(f32_to_act<ACT>(acc.y * inv)) << 16);
-  const uint32_t b = static_cast<uint32_t>(f32_to_act<ACT>(acc.z * inv)) |
-                     (static_cast<uint32_t>(f32_to_act<ACT>(acc.w * inv)) << 16);
-  *reinterpret_cast<uint2*>(orow + 4 * lane) = make_uint2(a, b);
 }
 
 // Query rows of a segment: a plain unit has its item's G query heads of KV
@@ -630,8 +624,8 @@ __device__ __forceinline__ void settle_partial(const Prm& prm, const Seg& s, int
     return (q == 0 && !a_inside) ? 2 * wk + 1 : 2 * wk;
   };
   auto out_of = [&](int r) { return row_offset<G>(prm, s, r); };
-  merge_unit_warp<ACT, R>(prm.partials, reinterpret_cast<uint16_t*>(prm.out), nslots, rows, slot_of,
-                          out_of, lane);
+  uint16_t* out = reinterpret_cast<uint16_t*>(prm.out);
+  merge_unit_warp<ACT, R>(prm.partials, out, nslots, rows, slot_of, out_of, lane);
   // every arrival is in: re-arm the counter for the next launch (no reply needed)
   if (lane == 0) asm volatile("st.relaxed.gpu.global.s32 [%0], 0;" ::"l"(prm.counters + wa) : "memory");
 }
@@ -1130,9 +1124,9 @@ __global__ void __launch_bounds__(kWarps * 32)
   Producer<KV> prod;
   Cursor cur;
   cur.init(prm, g0, g1, w);  // kernel parameters only: may overlap the previous kernel
+  prod.init(prm, cur);
   dev::grid_dep_wait();
   dev::grid_dep_launch();
-  prod.init(prm, cur);
 #pragma unroll 1
   for (int k = 0; k < T::kStages; ++k) prod.issue(prm, &tmk, &tmv, ring, bars, w, lane);
 
@@ -1169,25 +1163,59 @@ struct ReduceKParams {
   DecodePlan plan;
 };
 
-// Fixed partitions: CTA = (head, item), one warp per query row of the group;
-// each merges that row over the item's partitions (if there is more than one)
-// into the output.
+// Fixed partitions: CTA = (head, item, query row); its 4 warps merge a quarter
+// of the item's partitions each, then warp 0 combines the four partial merges
+// (shared memory) and writes the output row.  Items with a single partition
+// wrote their output directly.
 template <int ACT>
-__global__ void __launch_bounds__(kMaxGroup * 32) reduce_fixed_kernel(const __grid_constant__ ReduceKParams prm) {
+__global__ void __launch_bounds__(128) reduce_fixed_kernel(const __grid_constant__ ReduceKParams prm) {
   dev::grid_dep_wait();
   dev::grid_dep_launch();
   const DecodePlan& P = prm.plan;
-  const int h = blockIdx.x / P.n;
-  const int i = blockIdx.x - h * P.n;
+  const int row = blockIdx.x % prm.group;
+  const int hi = blockIdx.x / prm.group;
+  const int h = hi / P.n;
+  const int i = hi - h * P.n;
   const int np = P.pre[i + 1] - P.pre[i];
-  if (np <= 1) return;
+  if (np <= 1) return;  // uniform over the CTA
   const int64_t base = static_cast<int64_t>(h) * P.per_head + P.pre[i];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint16_t* obase = reinterpret_cast<uint16_t*>(prm.out) + i * prm.q_item_stride +
-                    (h * prm.group) * kHeadDim;
-  for (int gg = warp; gg < prm.group; gg += blockDim.x >> 5)
-    merge_row<ACT>(prm.partials, obase + gg * kHeadDim, gg, np,
-                   [&](int q) { return static_cast<int>(base + q); }, lane);
+  const int per = (np + 3) / 4;
+  const int kb = min(np, warp * per), ke = min(np, kb + per);
+  float M, L;
+  float4 acc;
+  merge_row_part(prm.partials, row, kb, ke, [&](int q) { return base + q; }, lane, M, L, acc);
+  __shared__ float s_m[4], s_l[4];
+  __shared__ float4 s_acc[4][32];
+  if (lane == 0) {
+    s_m[warp] = M;
+    s_l[warp] = L;
+  }
+  s_acc[warp][lane] = acc;
+  __syncthreads();
+  if (warp != 0) return;
+  float Mt = fmaxf(fmaxf(s_m[0], s_m[1]), fmaxf(s_m[2], s_m[3]));
+  const float ref = Mt == -INFINITY ? 0.f : Mt;
+  float Lt = 0.f;
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float wq = dev::exp2_approx(s_m[q] - ref);  // 0 for an empty quarter
+    const float4 x = s_acc[q][lane];
+    Lt += wq * s_l[q];
+    a.x += wq * x.x;
+    a.y += wq * x.y;
+    a.z += wq * x.z;
+    a.w += wq * x.w;
+  }
+  const float inv = 1.f / Lt;
+  uint16_t* orow = reinterpret_cast<uint16_t*>(prm.out) + i * prm.q_item_stride +
+                   (h * prm.group + row) * kHeadDim;
+  const uint32_t lo = static_cast<uint32_t>(f32_to_act<ACT>(a.x * inv)) |
+                      (static_cast<uint32_t>(f32_to_act<ACT>(a.y * inv)) << 16);
+  const uint32_t hi2 = static_cast<uint32_t>(f32_to_act<ACT>(a.z * inv)) |
+                       (static_cast<uint32_t>(f32_to_act<ACT>(a.w * inv)) << 16);
+  *reinterpret_cast<uint2*>(orow + 4 * lane) = make_uint2(lo, hi2);
 }
 
 // ================================================================== launchers
@@ -1305,10 +1333,10 @@ cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CU
   rp.group = args.group;
   rp.total = prm.total;
   std::memcpy(&rp.plan, &plan, sizeof(DecodePlan));
-  const int grid = plan.n * pool.num_kv_heads;
+  const int grid = plan.n * pool.num_kv_heads * args.group;
   e = pool.act_dtype == kBF16
-          ? launch_pdl(reduce_fixed_kernel<kBF16>, dim3(grid), dim3(32 * args.group), 0, stream, rp)
-          : launch_pdl(reduce_fixed_kernel<kFP16>, dim3(grid), dim3(32 * args.group), 0, stream, rp);
+          ? launch_pdl(reduce_fixed_kernel<kBF16>, dim3(grid), dim3(128), 0, stream, rp)
+          : launch_pdl(reduce_fixed_kernel<kFP16>, dim3(grid), dim3(128), 0, stream, rp);
   if (e == cudaSuccess) ++*launches;
   return e;
 }
