@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--separate-append", action="store_true",
+                    help="append with pa_append_kv and decode with pa_decode_attention (two launches "
+                         "per layer) instead of the fused pa_decode_attention_append")
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling: keep only the first N layers (a smaller case of the same "
                          "kernels; the JSON line then names the reduced workload)")
@@ -232,6 +235,7 @@ class Runner:
         self.torch, self.pa, self.w = torch, pa, w
         self.dev = device
         self.partition = partition
+        self.fused = True
         gen = torch.Generator(device=device)
         gen.manual_seed(1000 + seed)
         act = torch.bfloat16 if w.act_dtype == "bf16" else torch.float16
@@ -318,13 +322,18 @@ class Runner:
         scale = ctypes.c_float(w.scale)
         for layer in range(w.num_layers):
             pq, pk, pv, po = ptrs[layer]
-            st = L.pa_append_kv(self.pool.handle, layer, n, sp, pos, pk, pv, stream)
-            if st != 0:
-                raise RuntimeError(f"pa_append_kv: {self.pa.pa_last_error()}")
+            if not self.fused:
+                st = L.pa_append_kv(self.pool.handle, layer, n, sp, pos, pk, pv, stream)
+                if st != 0:
+                    raise RuntimeError(f"pa_append_kv: {self.pa.pa_last_error()}")
             if dec_events is not None:
                 dec_events[0].record()
-            st = L.pa_decode_attention(self.pool.handle, layer, n, sp, w.num_q_heads, pq, po, scale,
-                                       self.partition, stream)
+            if self.fused:   # append of the step's token and decode in one launch
+                st = L.pa_decode_attention_append(self.pool.handle, layer, n, sp, pk, pv, w.num_q_heads,
+                                                  pq, po, scale, self.partition, stream)
+            else:
+                st = L.pa_decode_attention(self.pool.handle, layer, n, sp, w.num_q_heads, pq, po, scale,
+                                           self.partition, stream)
             if dec_events is not None:
                 dec_events[1].record()
                 dec_events = None  # time the first layer's decode only
@@ -358,6 +367,7 @@ def run_ours(a, rank, world, local_rank):
     w = make_workload(a, a.seed + rank)
     partition = w.partition_tokens if a.partition is None else a.partition
     r = Runner(w, device, partition, a.seed + rank)
+    r.fused = not a.separate_append
     stream_obj = torch.cuda.current_stream(device)
     stream = ctypes.c_void_p(stream_obj.cuda_stream)
     pa = r.pa
@@ -455,7 +465,8 @@ def run_ours(a, rank, world, local_rank):
         "data": "synthetic (seeded N(0,1) K/V/Q, seeded lengths and block placement)",
         "config": {**describe(w, partition), "parallelism": f"replicas x{world} (no exchange step)"},
         "roofline": {
-            "kernel": "decode attention (decode kernel + split-KV reduce), first layer of each step",
+            "kernel": ("decode attention" + (" with the step's append fused" if r.fused else "") +
+                       " (decode kernel, + reduce kernel for fixed partitions), layer 0 of every 4th step"),
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peak,
@@ -476,6 +487,8 @@ def run_ours(a, rank, world, local_rank):
         "clocks": clk.summary(),
         "e2e": e2e,
     }
+    line["config"]["append"] = ("fused into the decode launch (pa_decode_attention_append)" if r.fused
+                                else "separate launch (pa_append_kv)")
     if w.name == "tiny":
         line["graph_batch"] = graph_batch(r, 1000)
     if rank == 0 and not a.no_cpu:

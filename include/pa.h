@@ -184,6 +184,22 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, int32_t n, const int
                               int32_t num_q_heads, const void *q, void *out, float scale,
                               int32_t partition_tokens, void *stream);
 
+/* pa_append_kv of each sequence's last token followed by pa_decode_attention,
+ * in one launch: the K/V rows k_new[i], v_new[i] (device [n][num_kv_heads]
+ * [head_dim] act_dtype) are written to position len(seqs[i]) - 1 -- the last
+ * slot reserved by pa_alloc_blocks -- and attended to in the same pass.  The
+ * worker that reads that slot's block writes the row into the cache and into
+ * its staged copy of the block, so the result (cache contents included) is
+ * exactly that of the two separate calls, with one launch fewer per layer.
+ * Each sequence may appear at most once; its last slot must lie in a block no
+ * other sequence shares (copy-on-write happens in pa_alloc_blocks).  Other
+ * arguments and errors as pa_decode_attention and pa_append_kv; a failure on
+ * the host launches nothing. */
+pa_status pa_decode_attention_append(pa_pool *pool, int32_t layer, int32_t n, const int32_t *seqs,
+                                     const void *k_new, const void *v_new, int32_t num_q_heads,
+                                     const void *q, void *out, float scale,
+                                     int32_t partition_tokens, void *stream);
+
 /* Decode attention for callers that cannot allocate device memory -- for
  * example a plugin or custom-operator interface of a serving engine that
  * reserves all free HBM for its own KV pool and hands a kernel only its input

@@ -32,6 +32,7 @@ from .binding import (  # noqa: F401
     pa_check_device_errors,
     pa_debug_fail_after,
     pa_decode_attention,
+    pa_decode_attention_append,
     pa_decode_attention_noalloc,
     pa_fork_cow,
     pa_free,

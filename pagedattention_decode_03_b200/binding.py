@@ -38,7 +38,7 @@ EXPORTS = (
     "pa_alloc_blocks_n", "pa_fork_cow", "pa_append_kv", "pa_decode_attention", "pa_free",
     "pa_get_seq", "pa_get_refcounts", "pa_get_free_list", "pa_get_cow_log", "pa_launch_count",
     "pa_check_device_errors", "pa_debug_fail_after", "pa_last_error", "pa_status_string",
-    "pa_decode_attention_noalloc", "pa_last_decode_plan",
+    "pa_decode_attention_noalloc", "pa_last_decode_plan", "pa_decode_attention_append",
 )
 
 
@@ -97,6 +97,8 @@ def lib() -> ctypes.CDLL:
         L.pa_fork_cow.argtypes = [vp, i32, i32]
         L.pa_append_kv.argtypes = [vp, i32, i32, _i32p, _i32p, vp, vp, vp]
         L.pa_decode_attention.argtypes = [vp, i32, i32, _i32p, i32, vp, vp, ctypes.c_float, i32, vp]
+        L.pa_decode_attention_append.argtypes = [vp, i32, i32, _i32p, vp, vp, i32, vp, vp, ctypes.c_float,
+                                                 i32, vp]
         L.pa_decode_attention_noalloc.argtypes = [ctypes.POINTER(pa_pool_desc), i32, i32, vp, _i32p,
                                                   i32, vp, vp, ctypes.c_float, vp]
         L.pa_free.argtypes = [vp, i32]
@@ -307,6 +309,22 @@ def pa_decode_attention(pool: Pool, layer: int, seqs, q, out, scale: float,
     _check(lib().pa_decode_attention(pool.handle, layer, n, _ptr(s), hq, ctypes.c_void_p(qp),
                                      ctypes.c_void_p(op), ctypes.c_float(scale),
                                      partition_tokens, _stream(stream)), "pa_decode_attention")
+
+
+def pa_decode_attention_append(pool: Pool, layer: int, seqs, k_new, v_new, q, out, scale: float,
+                               partition_tokens: int = 0, stream=None) -> None:
+    """Append each sequence's last token (k_new/v_new [n][H_kv][128]) and decode, in one launch."""
+    s = _i32(seqs)
+    n = len(s)
+    hq = q.shape[1] if q.dim() == 3 else -1
+    kp = _dev_tensor(k_new, "k_new", n, pool.num_kv_heads, pool.act_dtype)
+    vp = _dev_tensor(v_new, "v_new", n, pool.num_kv_heads, pool.act_dtype)
+    qp = _dev_tensor(q, "q", n, hq, pool.act_dtype)
+    op = _dev_tensor(out, "out", n, hq, pool.act_dtype)
+    _check(lib().pa_decode_attention_append(pool.handle, layer, n, _ptr(s), ctypes.c_void_p(kp),
+                                            ctypes.c_void_p(vp), hq, ctypes.c_void_p(qp),
+                                            ctypes.c_void_p(op), ctypes.c_float(scale), partition_tokens,
+                                            _stream(stream)), "pa_decode_attention_append")
 
 
 def pa_decode_attention_noalloc(desc: pa_pool_desc, layer: int, block_tables, seq_lens, q, out,

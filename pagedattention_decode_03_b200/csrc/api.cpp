@@ -493,10 +493,13 @@ pa_status pa_append_kv(pa_pool* p, int32_t layer, int32_t T, const int32_t* seqs
   return PA_OK;
 }
 
-pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
-                              int32_t num_q_heads, const void* q, void* out, float scale,
-                              int32_t partition_tokens, void* stream) {
-  g_last_error.clear();
+namespace {
+
+// pa_decode_attention, and with k_new / v_new the fused append of
+// pa_decode_attention_append (validated by the caller).
+pa_status decode_call(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
+                      int32_t num_q_heads, const void* q, void* out, float scale,
+                      int32_t partition_tokens, void* stream, const void* k_new, const void* v_new) {
   if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
   if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
   if (layer < 0 || layer >= p->d.num_layers) return fail(PA_ERR_INVALID_ARG, "layer out of range");
@@ -545,6 +548,8 @@ pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_
   const int cap = pa::decode_worker_capacity(p->d.kv_dtype, group, p->num_sms);
   const int64_t slots_cap = p->view.partial_slots;
   pa::DecodeArgs args;
+  args.k_new = k_new;
+  args.v_new = v_new;
   args.q = q;
   args.out = out;
   args.layer = layer;
@@ -602,7 +607,25 @@ pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_
     static thread_local pa::SibPlan sib;
     if (mode == pa::kSplitStreamK && group <= 4 &&
         build_sib_plan(p, seqs + at, cnt, group, cap, sib, p->order, p->set_of)) {
+      if (k_new != nullptr) {
+        // Sibling sets put several sequences' last blocks back to back in one
+        // worker's share; that worker's row patches would run in series, so the
+        // rows go in with the append kernel instead (same cache contents).
+        p->slots.resize(cnt);
+        for (int32_t t = 0; t < cnt; ++t)
+          p->bm->slot(seqs[at + t], p->bm->len(seqs[at + t]) - 1, &p->slots[t]);
+        const size_t row = static_cast<size_t>(p->d.num_kv_heads) * pa::kHeadDim * 2;
+        int al = 0;
+        e = pa::launch_append(p->view, layer, p->slots.data(), cnt,
+                              static_cast<const uint8_t*>(k_new) + at * row,
+                              static_cast<const uint8_t*>(v_new) + at * row, nullptr, nullptr, 0, s, &al);
+        p->launches += al;
+        if (e != cudaSuccess) return cuda_fail(e, "append launch");
+        args.k_new = args.v_new = nullptr;
+      }
       e = pa::launch_decode_sib(p->view, &p->tmk, &p->tmv, sib, args, s, &launches);
+      args.k_new = k_new;
+      args.v_new = v_new;
       p->last_sets += sib.sets;
       p->last_tiles += (sib.per_head - static_cast<int64_t>(sib.alpha) * sib.nu) * H;
     } else {
@@ -614,6 +637,47 @@ pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_
     at += cnt;
   }
   return PA_OK;
+}
+
+}  // namespace
+
+pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
+                              int32_t num_q_heads, const void* q, void* out, float scale,
+                              int32_t partition_tokens, void* stream) {
+  g_last_error.clear();
+  return decode_call(p, layer, n, seqs, num_q_heads, q, out, scale, partition_tokens, stream,
+                     nullptr, nullptr);
+}
+
+pa_status pa_decode_attention_append(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
+                                     const void* k_new, const void* v_new, int32_t num_q_heads,
+                                     const void* q, void* out, float scale,
+                                     int32_t partition_tokens, void* stream) {
+  g_last_error.clear();
+  if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
+  if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
+  if (layer < 0 || layer >= p->d.num_layers) return fail(PA_ERR_INVALID_ARG, "layer out of range");
+  if (n < 0 || (n > 0 && (!seqs || !k_new || !v_new))) return fail(PA_ERR_INVALID_ARG, "null argument");
+  if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & 15)
+    return fail(PA_ERR_INVALID_ARG, "k_new / v_new must be 16-byte aligned");
+  // the target slot of every item: the last reserved position of its sequence,
+  // in a block no other sequence shares; each sequence at most once
+  p->a.assign(n, 0);
+  std::vector<int32_t>& seen = p->b;
+  seen.assign(p->d.max_seqs, 0);
+  for (int32_t i = 0; i < n; ++i) {
+    pa_status st = seq_arg(p, seqs[i]);
+    if (st != PA_OK) return st;
+    if (!p->bm->active(seqs[i])) return fail(PA_ERR_NO_SEQ, "pa_decode_attention_append: no such sequence");
+    if (seen[seqs[i]]++) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention_append: a sequence named twice");
+    const int32_t len = p->bm->len(seqs[i]);
+    if (len < 1) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention_append: empty sequence");
+    int64_t slot = 0;
+    st = bm_status(p->bm->slot(seqs[i], len - 1, &slot), "pa_decode_attention_append");
+    if (st != PA_OK) return st;
+  }
+  return decode_call(p, layer, n, seqs, num_q_heads, q, out, scale, partition_tokens, stream, k_new,
+                     v_new);
 }
 
 pa_status pa_get_seq(pa_pool* p, int32_t seq, int32_t* len, int32_t* table, int32_t cap,

@@ -68,6 +68,15 @@ struct DecodeKParams {
   float scale;
   int32_t layer, num_kv_heads, num_blocks, mbps, group;
   int64_t total;           // work units over all heads
+  // Fused append (null k_new: none): the K/V rows of each item's last token,
+  // [n][H][128] act dtype, written into the cache by the worker that reads the
+  // item's last block, which also patches them into its staged tile.
+  const uint8_t* k_new;
+  const uint8_t* v_new;
+  uint8_t* k_cache;
+  uint8_t* v_cache;
+  const float* k_inv;
+  const float* v_inv;
   PlanT plan;
 };
 
@@ -89,6 +98,7 @@ struct Seg {
 struct BlockRef {
   int32_t seq, b, len;
   uint32_t cols;  // bit r set: query row r takes part (all 8 for plain units)
+  int32_t item;   // the item whose table row this is
 };
 
 __device__ __forceinline__ int n_entries(const DecodePlan& P) { return P.n; }
@@ -243,13 +253,13 @@ __device__ __forceinline__ Seg next_seg(const DecodeKParams<SibPlan>& prm, int64
 // member order, each taken only by that member's G rows.
 template <int G>
 __device__ __forceinline__ BlockRef locate(const DecodeKParams<DecodePlan>&, const Seg& s, int o) {
-  return BlockRef{s.seq, o, s.len, 0xffu};
+  return BlockRef{s.seq, o, s.len, 0xffu, s.i};
 }
 template <int G>
 __device__ __forceinline__ BlockRef locate(const DecodeKParams<SibPlan>& prm, const Seg& s, int o) {
   const SibPlan& P = prm.plan;
   const int cp = P.cp[s.k];
-  if (o < cp) return BlockRef{s.seq, o, s.len, 0xffu};
+  if (o < cp) return BlockRef{s.seq, o, s.len, 0xffu, s.i};
   const int m0 = P.mem0[s.k], m = P.mem0[s.k + 1] - m0;
   int j = 0, item = s.i;
   for (int jj = 1; jj < m; ++jj) {
@@ -259,7 +269,7 @@ __device__ __forceinline__ BlockRef locate(const DecodeKParams<SibPlan>& prm, co
     item = it;
   }
   return BlockRef{P.seq[item], cp + (o - P.part[item]), P.len[item],
-                  ((1u << G) - 1u) << (j * G)};
+                  ((1u << G) - 1u) << (j * G), item};
 }
 
 // The segments of one worker, in processing order.  Stream-K: a worker's last
@@ -324,6 +334,20 @@ struct Cursor {
   }
 };
 
+// ------------------------------------------------------ fused append rows
+__device__ __forceinline__ bool is_last_block(const BlockRef& br) { return br.b == (br.len - 1) / kBlock; }
+
+// Address of this lane's 16 bytes of the rows.  (Calls whose plan has sibling
+// sets append with the append kernel instead: a set puts several sequences'
+// last blocks into one worker's share, and their row loads would run in
+// series.)
+template <class Prm>
+__device__ __forceinline__ const uint4* new_row_ptr(const Prm& prm, int h, int item, int lane) {
+  const int64_t src_el = (static_cast<int64_t>(item) * prm.num_kv_heads + h) * kHeadDim + (lane & 15) * 8;
+  return reinterpret_cast<const uint4*>((lane < 16 ? prm.k_new : prm.v_new) + src_el * 2);
+}
+
+
 // ------------------------------------------------------------------ producer
 template <int KV>
 struct Producer {
@@ -332,6 +356,7 @@ struct Producer {
   int32_t b;          // next block of seg to fetch
   int32_t tc_val, tc_base, tc_unit;
   uint32_t issued;
+  int32_t* phys_s;    // shared memory: physical block id of each stage
 
   // Starts from a copy of the consumer's cursor (same segments, same order).
   template <class Prm>
@@ -371,6 +396,7 @@ struct Producer {
     }
     const uint32_t stage = issued % Tile<KV>::kStages;
     const uint32_t bar = bars + stage * 8;
+    if (lane == 0) phys_s[stage] = phys;
     const uint32_t dst = ring + stage * Tile<KV>::kStageBytes;
     const int32_t row =
         ((prm.layer * prm.num_blocks + phys) * prm.num_kv_heads + seg.h) * kBlock;
@@ -1061,9 +1087,50 @@ template <int KV, int ACT, int G>
 using PathFor = typename std::conditional<(G >= 4), MmaPath<KV, ACT, G>, FmaPath<KV, ACT, G>>::type;
 
 // ===================================================================== kernel
+// Fused append: the K/V rows of `item`'s last token (position len-1) for KV
+// head h.  Lane l < 16 carries elements 8l .. 8l+7 of the K row, lane 16 + l
+// those of the V row (act dtype, 16 bytes).
+// Write those rows into the cache slot of physical block `phys` and into row
+// (len-1) % 16 of the staged K and V tiles (the copy brought the block in
+// before the row was written).  Same values as the append kernel: 16-bit rows
+// are copied; FP8 codes are E4M3(rn, satfinite)(fp32(x) * inv_scale).
+template <int KV, int ACT, class Prm>
+__device__ __forceinline__ void append_last_token(const Prm& prm, int h, int len, int32_t phys,
+                                                  uint8_t* st, uint4 val, int lane) {
+  using T = Tile<KV>;
+  const int r = (len - 1) % kBlock;
+  const int kv = lane >> 4, c = lane & 15;
+  uint8_t* tile = st + kv * T::kBytes;
+  uint8_t* cache = kv ? prm.v_cache : prm.k_cache;
+  const int64_t dst_el =
+      ((static_cast<int64_t>(prm.layer) * prm.num_blocks + phys) * prm.num_kv_heads + h) * kBlock * kHeadDim +
+      static_cast<int64_t>(r) * kHeadDim;
+  if constexpr (KV == kFP8) {
+    const float inv = (kv ? prm.v_inv : prm.k_inv)[prm.layer * prm.num_kv_heads + h];
+    const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+    uint32_t code[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float x0 = act_to_f32<ACT>(w[2 * k] & 0xffff), x1 = act_to_f32<ACT>(w[2 * k] >> 16);
+      const float x2 = act_to_f32<ACT>(w[2 * k + 1] & 0xffff), x3 = act_to_f32<ACT>(w[2 * k + 1] >> 16);
+      code[k] = static_cast<uint32_t>(dev::f32x2_to_e4m3x2(__fmul_rn(x0, inv), __fmul_rn(x1, inv))) |
+                (static_cast<uint32_t>(dev::f32x2_to_e4m3x2(__fmul_rn(x2, inv), __fmul_rn(x3, inv))) << 16);
+    }
+    const uint2 codes = make_uint2(code[0], code[1]);  // elements 8c .. 8c+7, one byte each
+    *reinterpret_cast<uint2*>(tile + r * 128 + (((c >> 1) ^ (r & 7)) << 4) + (c & 1) * 8) = codes;
+    dev::fence_proxy_async_smem();  // the stage's next copy overwrites these bytes
+    *reinterpret_cast<uint2*>(cache + dst_el + c * 8) = codes;
+  } else {
+    *reinterpret_cast<uint4*>(tile + (c >> 3) * 2048 + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = val;
+    dev::fence_proxy_async_smem();  // the stage's next copy overwrites these bytes
+    *reinterpret_cast<uint4*>(cache + (dst_el + c * 8) * 2) = val;
+  }
+  __syncwarp();  // the staged row is complete before any lane reads the tile
+}
+
 // One segment: wait for each staged block in turn, compute on it, and refill
 // the freed stage with the worker's next block.  False if a wait gave up.
-template <int KV, int G, class Path, class Prm>
+template <int KV, int ACT, int G, class Path, class Prm>
 __device__ __forceinline__ bool consume_segment(Path& path, const Prm& prm, const Seg& s,
                                                 Producer<KV>& prod, const CUtensorMap* tmk,
                                                 const CUtensorMap* tmv, uint8_t* ring_ptr,
@@ -1083,6 +1150,11 @@ __device__ __forceinline__ bool consume_segment(Path& path, const Prm& prm, cons
     const int nvalid = max(0, min(kBlock, br.len - br.b * kBlock));
     uint8_t* st = ring_ptr + stage * T::kStageBytes;
     if (nvalid < kBlock) zero_tail_rows<KV>(st + T::kBytes, nvalid, lane);
+    if constexpr (!kSibParams<Prm>) {  // sibling plans never carry a fused append
+      if (prm.k_new != nullptr && is_last_block(br))
+        append_last_token<KV, ACT>(prm, s.h, br.len, prod.phys_s[stage], st,
+                                   __ldcg(new_row_ptr(prm, s.h, br.item, lane)), lane);
+    }
     path.block(ring + stage * T::kStageBytes, ring + stage * T::kStageBytes + T::kBytes, nvalid,
                br.cols, lane);
     __syncwarp();
@@ -1111,6 +1183,8 @@ __global__ void __launch_bounds__(kWarps * 32)
   uint8_t* ring_ptr = smem + warp * T::kRingBytes;
   const uint32_t ring = dev::smem_u32(ring_ptr);
   const uint32_t bars = dev::smem_u32(smem + kWarps * T::kRingBytes) + warp * T::kStages * 8;
+  int32_t* phys_s = reinterpret_cast<int32_t*>(smem + kWarps * T::kRingBytes + kWarps * T::kStages * 8) +
+                    warp * T::kStages;
   if (lane == 0) {
     dev::tma_prefetch_desc(&tmk);
     dev::tma_prefetch_desc(&tmv);
@@ -1122,6 +1196,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int64_t g0 = worker_start(prm.total, w, W);
   const int64_t g1 = worker_start(prm.total, w + 1, W);
   Producer<KV> prod;
+  prod.phys_s = phys_s;
   Cursor cur;
   cur.init(prm, g0, g1, w);  // kernel parameters only: may overlap the previous kernel
   prod.init(prm, cur);
@@ -1140,7 +1215,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     const Seg s = cur.next(prm);
     if (!s.valid) break;
     const bool ok =
-        consume_segment<KV, G>(path, prm, s, prod, &tmk, &tmv, ring_ptr, ring, bars, consumed, w, lane);
+        consume_segment<KV, ACT, G>(path, prm, s, prod, &tmk, &tmv, ring_ptr, ring, bars, consumed, w, lane);
     if (!ok) {
       failed = true;
       break;
@@ -1221,7 +1296,8 @@ __global__ void __launch_bounds__(128) reduce_fixed_kernel(const __grid_constant
 // ================================================================== launchers
 template <int KV>
 constexpr size_t smem_bytes() {
-  return 1024 + kWarps * Tile<KV>::kRingBytes + kWarps * Tile<KV>::kStages * 8;
+  // rings, one mbarrier per stage, the physical block id of each staged block
+  return 1024 + kWarps * Tile<KV>::kRingBytes + kWarps * Tile<KV>::kStages * (8 + 4);
 }
 
 template <int KV, int ACT, int G, class PlanT>
@@ -1290,6 +1366,14 @@ void fill_params(DecodeKParams<PlanT>& prm, const PoolView& pool, const PlanT& p
   // q / out of this launch start at item_offset
   prm.q += static_cast<int64_t>(args.item_offset) * args.q_item_stride * 2;
   prm.out += static_cast<int64_t>(args.item_offset) * args.q_item_stride * 2;
+  // fused append: new rows [n][H][128] act dtype, from item_offset on
+  const int64_t kv_off = static_cast<int64_t>(args.item_offset) * pool.num_kv_heads * kHeadDim * 2;
+  prm.k_new = args.k_new ? static_cast<const uint8_t*>(args.k_new) + kv_off : nullptr;
+  prm.v_new = args.v_new ? static_cast<const uint8_t*>(args.v_new) + kv_off : nullptr;
+  prm.k_cache = static_cast<uint8_t*>(pool.k_cache);
+  prm.v_cache = static_cast<uint8_t*>(pool.v_cache);
+  prm.k_inv = pool.k_inv;
+  prm.v_inv = pool.v_inv;
 }
 
 template <class PlanT>

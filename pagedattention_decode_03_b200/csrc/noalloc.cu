@@ -221,6 +221,7 @@ extern "C" pa_status pa_decode_attention_noalloc(const pa_pool_desc* d, int32_t 
   plan.per_head = work;
   plan.workers = static_cast<int32_t>(std::max<int64_t>(1, W));
   pa::DecodeArgs args;
+  args.k_new = args.v_new = nullptr;
   args.q = q;
   args.out = out;
   args.layer = layer;

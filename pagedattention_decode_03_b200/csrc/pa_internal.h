@@ -125,6 +125,8 @@ struct DecodeArgs {
   float scale;            // softmax scale
   int64_t q_item_stride;  // elements between consecutive items of q / out (num_q_heads*128)
   int32_t item_offset;    // index of plan item 0 within the caller's arrays
+  const void* k_new;      // fused append: [n][H_kv][128] rows of each item's last token,
+  const void* v_new;      // or null (no append)
 };
 
 // Stream-K cost positions per work unit, in KV blocks: they stand for the

@@ -128,6 +128,19 @@ class Pair:
         pa.pa_decode_attention(self.pool, layer, seqs, q, out, w.scale, partition_tokens)
         return q_bits, out
 
+    def append_decode(self, step, layer, seqs, positions, partition_tokens=0):
+        """The step's append of every sequence's last token and the decode in one
+        call (pa_decode_attention_append); the oracle appends the same rows."""
+        w = self.w
+        k, v = step_kv_bits(w, step, layer)
+        q_bits = step_q_bits(w, step, layer)
+        q = to_dev(q_bits, w.act_dtype)
+        out = torch.empty_like(q)
+        pa.pa_decode_attention_append(self.pool, layer, seqs, to_dev(k, w.act_dtype),
+                                      to_dev(v, w.act_dtype), q, out, w.scale, partition_tokens)
+        self.append(layer, seqs, positions, k, v, gpu=False)
+        return q_bits, out
+
     def oracle_attention(self, layer, seqs, q_bits):
         ks = vs = None
         if self.scales is not None:
