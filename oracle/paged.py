@@ -26,7 +26,7 @@ What the pages define, and how this model reads it:
   into a contiguous buffer first, which is the plain definition the fused
   kernel must reproduce.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * free list is FIFO: allocate from the head, release to the tail, in
   logical-block order; its initial order is given by the caller;

@@ -28,12 +28,13 @@ def test_bytes_per_token_printed(printed):
         if "mib" in row:
             assert got / 2**20 == row["mib"], row["cite"]
         if "approx_mb" in row:
-            # the page rounds 524,288 B to "about 0.5 MB"
+            # the page rounds 524,288 B to half a megabyte
             assert got == 524288 and abs(got / 2**20 - row["approx_mb"]) < 1e-12, row["cite"]
 
 
 def test_bytes_per_token_ratios():
-    # GQA versus MHA at 64 KV heads: 8x ("That 8x footprint gap comes from KV-head sharing")
+    # GQA versus MHA at 64 KV heads: the per-token footprint differs by the KV-head
+    # ratio, 8x ("Managing the KV Cache", Reproduce Bytes per Token)
     gqa = sizing.kv_bytes_per_token(80, 8, 128, 2)
     mha = sizing.kv_bytes_per_token(80, 64, 128, 2)
     assert mha == 8 * gqa
