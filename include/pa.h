@@ -260,6 +260,18 @@ uint64_t pa_launch_count(const pa_pool *pool);
  * once for all of them (up to 8 / G sequences per set), so *kv_tiles can be
  * below the sum over sequences.  Either pointer may be NULL. */
 pa_status pa_last_decode_plan(const pa_pool *pool, int32_t *shared_sets, int64_t *kv_tiles);
+/* The sibling sets pa_decode_attention (partition_tokens = 0) would form for
+ * the n sequences `seqs` with query group `group` (1, 2, 4 or 8), from the
+ * host block tables alone (no device work; works on host-only pools too).
+ * set_of[i] = set of item i or -1; set_cp[k] = full blocks set k reads once
+ * (set_cp needs room for n entries); *n_sets = number of sets.  Sequences are
+ * ordered by their block tables and consecutive ones whose tables start with
+ * the same run of >= 2 full blocks are grouped, at most 8 / group per set;
+ * every member keeps at least its last block to itself.
+ * Errors: PA_ERR_INVALID_ARG (n above 512, bad group or sequence id),
+ * PA_ERR_NO_SEQ. */
+pa_status pa_plan_siblings(const pa_pool *pool, int32_t n, const int32_t *seqs, int32_t group,
+                           int32_t *set_of, int32_t *set_cp, int32_t *n_sets);
 
 /* Synchronise `stream`, read the device error word, clear it, and store the
  * PA_DEVERR_* bits in *bits.  Returns PA_ERR_DEVICE_CHECK if any bit was set,

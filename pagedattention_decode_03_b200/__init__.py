@@ -40,6 +40,7 @@ from .binding import (  # noqa: F401
     pa_get_free_list,
     pa_get_refcounts,
     pa_last_decode_plan,
+    pa_plan_siblings,
     pa_get_seq,
     pa_last_error,
     pa_launch_count,

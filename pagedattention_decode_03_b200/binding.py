@@ -39,6 +39,7 @@ EXPORTS = (
     "pa_get_seq", "pa_get_refcounts", "pa_get_free_list", "pa_get_cow_log", "pa_launch_count",
     "pa_check_device_errors", "pa_debug_fail_after", "pa_last_error", "pa_status_string",
     "pa_decode_attention_noalloc", "pa_last_decode_plan", "pa_decode_attention_append",
+    "pa_plan_siblings",
 )
 
 
@@ -109,6 +110,7 @@ def lib() -> ctypes.CDLL:
         L.pa_launch_count.argtypes = [vp]
         L.pa_launch_count.restype = ctypes.c_uint64
         L.pa_last_decode_plan.argtypes = [vp, _i32p, ctypes.POINTER(ctypes.c_int64)]
+        L.pa_plan_siblings.argtypes = [vp, i32, _i32p, i32, _i32p, _i32p, _i32p]
         L.pa_check_device_errors.argtypes = [vp, vp, u32p]
         L.pa_debug_fail_after.argtypes = [vp, i32]
         L.pa_last_error.argtypes = []
@@ -384,6 +386,18 @@ def pa_get_cow_log(pool: Pool):
 
 def pa_launch_count(pool: Pool) -> int:
     return int(lib().pa_launch_count(pool.handle))
+
+
+def pa_plan_siblings(pool: Pool, seqs, group: int) -> tuple[list, list]:
+    """(set of each item or -1, shared full blocks of each set) the decode would use."""
+    s = _i32(seqs)
+    n = len(s)
+    set_of = np.zeros(max(n, 1), np.int32)
+    set_cp = np.zeros(max(n, 1), np.int32)
+    ns = ctypes.c_int32()
+    _check(lib().pa_plan_siblings(pool.handle, n, _ptr(s), group, _ptr(set_of), _ptr(set_cp),
+                                  ctypes.byref(ns)), "pa_plan_siblings")
+    return set_of[:n].tolist(), set_cp[: ns.value].tolist()
 
 
 def pa_last_decode_plan(pool: Pool) -> tuple[int, int]:

@@ -729,6 +729,31 @@ pa_status pa_get_cow_log(pa_pool* p, int32_t* pairs, int32_t cap, int32_t* n) {
 
 uint64_t pa_launch_count(const pa_pool* p) { return p ? p->launches : 0; }
 
+pa_status pa_plan_siblings(const pa_pool* p, int32_t n, const int32_t* seqs, int32_t group,
+                           int32_t* set_of, int32_t* set_cp, int32_t* n_sets) {
+  g_last_error.clear();
+  if (!p || (n > 0 && (!seqs || !set_of || !set_cp)) || !n_sets)
+    return fail(PA_ERR_INVALID_ARG, "null argument");
+  if (n < 0 || n > pa::kDecodeItemsCap)
+    return fail(PA_ERR_INVALID_ARG, "n must be in [0, 512] (one launch's items)");
+  if (group != 1 && group != 2 && group != 4 && group != 8)
+    return fail(PA_ERR_INVALID_ARG, "group must be 1, 2, 4 or 8");
+  for (int32_t i = 0; i < n; ++i) {
+    pa_status st = seq_arg(p, seqs[i]);
+    if (st != PA_OK) return st;
+    if (!p->bm->active(seqs[i])) return fail(PA_ERR_NO_SEQ, "pa_plan_siblings: no such sequence");
+    if (p->bm->len(seqs[i]) < 1) return fail(PA_ERR_INVALID_ARG, "pa_plan_siblings: empty sequence");
+  }
+  static thread_local pa::SibPlan sp;
+  std::vector<int32_t> order, set_idx;
+  int32_t sets = 0;
+  if (build_sib_plan(p, seqs, n, group, pa::kMaxWorkers, sp, order, set_idx)) sets = sp.sets;
+  for (int32_t i = 0; i < n; ++i) set_of[i] = sets ? set_idx[i] : -1;
+  for (int32_t k = 0; k < sets; ++k) set_cp[k] = sp.cp[k];
+  *n_sets = sets;
+  return PA_OK;
+}
+
 pa_status pa_check_device_errors(pa_pool* p, void* stream, uint32_t* bits) {
   g_last_error.clear();
   if (!p || !bits) return fail(PA_ERR_INVALID_ARG, "null argument");
