@@ -21,15 +21,27 @@
 //     16 tokens of a block on M and the (padded) query group on N; S^T stays in
 //     registers, the online softmax runs on the accumulator fragments, and P^T
 //     reaches the PV MMA through movmatrix.  G <= 2: fp32 FMAs on CUDA cores.
-//   * Work is spread over all warps of the GPU in equal shares of KV blocks
-//     (stream-K style): a worker's share can start and end inside a sequence;
-//     partial results (running max m, sum l, unnormalised o) of a cut
-//     sequence are merged by log-sum-exp inside the kernel, by the last of its
-//     workers to finish.  Fixed-size partitions (merged by a separate
-//     reduction kernel) and "never split" are the two other modes.
+//   * Work is spread over all warps of the GPU in equal shares of a work axis
+//     that lists each unit's KV blocks after a few "cost positions" standing
+//     for the unit's fixed segment cost (stream-K style): a worker's share can
+//     start and end inside a sequence; partial results (running max m, sum l,
+//     unnormalised o) of a cut sequence are merged by log-sum-exp inside the
+//     kernel, by the last of its workers to finish.  Fixed-size partitions
+//     (merged by a separate reduction kernel) and "never split" are the two
+//     other modes.
+//   * Forks of one prompt share its blocks by reference count ("Managing the
+//     KV Cache", Block Tables and Sharing); a sibling set is one unit whose
+//     common blocks are read once for all members' query rows, followed by
+//     each member's own blocks with the other members' rows masked.
+//   * The step's append may ride along: the worker that reads a sequence's
+//     last block writes the new K/V row into the cache and into its staged
+//     tile before computing on it.
 //   * FP8 E4M3 KV: tiles are half the bytes; codes are converted to f16 with
 //     the hardware cvt (exact), K's scale is folded into the logit scale and
 //     V's into the output.
+//   * Launched with programmatic stream serialization: the parameter-only
+//     prologue overlaps the previous kernel, which is waited for before any
+//     memory access.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
