@@ -87,3 +87,41 @@ def test_fused_host_errors_launch_nothing():
     assert e.value.status == pa.PA_ERR_INVALID_ARG
     assert pa.pa_launch_count(p.pool) == n0
     p.check_metadata()
+
+
+def test_fused_gqa8b_full_size():
+    """The benchmark's step at full size: 64 sequences of 128..4096 tokens,
+    append fused into the decode, growth across block boundaries; every 5th
+    step checked in full (cache bit-exact, every output within tolerance)."""
+    w = workload("gqa8b", steps=11)
+    p = Pair(w)
+    p.prefill()
+    for step in range(w.steps):
+        seqs, pos = p.reserve_step(step)
+        q, out = p.append_decode(step, 0, seqs, pos, 0)
+        if step % 5 == 0:
+            p.check_metadata()
+            p.check_cache(0)
+            p.check_attention(0, seqs, q, out)
+    assert p.device_errors() == 0
+
+
+def test_fused_gqa70b_layers():
+    """80 layers on the 2,491-block pool, every layer's append fused into its
+    decode as in the benchmark step; layers 0 and 79 carry data and are
+    compared at steps 1, 8 and 16 (layer 0 at every step)."""
+    w = workload("gqa70b_headroom")
+    layers = [0, 79]
+    p = Pair(w, layers=layers)
+    p.prefill(gpu_layers=layers)
+    for step in range(w.steps):
+        seqs, pos = p.reserve_step(step)
+        for layer in range(w.num_layers):
+            q, out = p.append_decode(step, layer, seqs, pos, 0)
+            if layer in layers and (layer == 0 or step in (0, 7, 15)):
+                p.check_attention(layer, seqs, q, out)
+        if step in (0, 7, 15):
+            p.check_metadata()
+            for layer in layers:
+                p.check_cache(layer)
+    assert p.device_errors() == 0
