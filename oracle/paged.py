@@ -36,6 +36,31 @@ Readings where the pages are silent:
 * the copy-on-write copy covers the whole block for every layer, K and V;
 * a query of head i attends through KV head floor(i / G), G = H_q / H_kv;
 * no mask beyond the sequence length; the scale is a caller argument.
+
+Block-granular prefix caching (kv-cache-pagedattention-serving, Beyond
+paging: radix trees and continuous batching; "Managing the KV Cache", Block
+Tables and Sharing and Answer Key item 4): a full block whose KV the caller
+has written may be registered under the token prefix it ends, i.e. all
+tokens from the sequence start to the block's last slot (the KV of a token
+depends on every token before it).  A new prompt reuses, from its first
+block on, each full block whose whole prefix is registered, and stops at the
+first one that is not; so a 103-token prompt reuses at most 96 tokens with
+16-token blocks.  Registered blocks stay reference counted; when no sequence
+references one it is kept, with its contents, on a least-recently-used list
+and is evicted only when a block is needed and the free list is empty.
+Readings where the pages are silent:
+
+* a registered block is immutable: writing a slot of it is refused like a
+  write into a shared block;
+* the first registration of a prefix wins; registering another block with
+  the same prefix leaves that block unregistered;
+* when a release drops several registered blocks to zero references, they
+  join the recently-used end in reverse logical order, so a longer prefix
+  is evicted before the shorter prefix it extends (a block is only reached
+  through its predecessors);
+* a prompt whose every token falls in registered blocks reuses all of them
+  (whether the last token is recomputed to get logits is a scheduler's
+  choice, outside the pool).
 """
 from __future__ import annotations
 
@@ -84,6 +109,11 @@ class PagedKVOracle:
         self.tables: dict[int, list[int]] = {}
         self.lens: dict[int, int] = {}
         self.cow_log: list[tuple[int, int]] = []
+        # prefix cache: whole-token-prefix tuple -> block, block -> prefix, and
+        # the registered blocks nothing references, least recently used first
+        self.registry: dict[tuple, int] = {}
+        self.key_of: dict[int, tuple] = {}
+        self.cached: collections.OrderedDict[int, None] = collections.OrderedDict()
         layers = range(num_layers) if stored_layers is None else stored_layers
         store = np.uint8 if kv_dtype == "fp8_e4m3" else np.uint16
         shape = (num_blocks, num_kv_heads, block_size, head_dim)
@@ -101,12 +131,12 @@ class PagedKVOracle:
             return Status.INVALID_ARG
         cow = new_len > cur and cur % self.B != 0 and self.ref[table[-1]] > 1
         grow = _ceil_div(new_len, self.B) - len(table)
-        if int(cow) + grow > len(self.free):
+        if int(cow) + grow > len(self.free) + len(self.cached):
             return Status.NO_BLOCKS
         table = list(table)
         if cow:
             src = table[-1]
-            dst = self.free.popleft()
+            dst = self._take()
             for layer in self.k:
                 self.k[layer][dst] = self.k[layer][src]
                 self.v[layer][dst] = self.v[layer][src]
@@ -115,12 +145,21 @@ class PagedKVOracle:
             table[-1] = dst
             self.cow_log.append((src, dst))
         for _ in range(grow):
-            b = self.free.popleft()
+            b = self._take()
             self.ref[b] = 1
             table.append(b)
         self.tables[seq] = table
         self.lens[seq] = new_len
         return Status.OK
+
+    def _take(self) -> int:
+        """A block for new contents: the free list's head, else the least
+        recently used cached block, which then leaves the prefix registry."""
+        if self.free:
+            return self.free.popleft()
+        b, _ = self.cached.popitem(last=False)
+        del self.registry[self.key_of.pop(b)]
+        return b
 
     def fork(self, parent: int, child: int) -> Status:
         """`child` shares every block of `parent` (reference count + 1)."""
@@ -137,13 +176,17 @@ class PagedKVOracle:
         return Status.OK
 
     def release(self, seq: int) -> Status:
-        """Drop `seq`; blocks whose count reaches zero return to the free tail."""
+        """Drop `seq`; blocks whose count reaches zero return to the free tail,
+        registered ones to the recently-used end of the cached list instead."""
         if seq not in self.tables:
             return Status.NO_SEQ if 0 <= seq < self.max_seqs else Status.INVALID_ARG
         for b in self.tables[seq]:
             self.ref[b] -= 1
-            if self.ref[b] == 0:
+            if self.ref[b] == 0 and b not in self.key_of:
                 self.free.append(b)
+        for b in reversed(self.tables[seq]):
+            if self.ref[b] == 0 and b in self.key_of:
+                self.cached[b] = None
         del self.tables[seq]
         del self.lens[seq]
         return Status.OK
@@ -155,9 +198,70 @@ class PagedKVOracle:
         if not 0 <= pos < self.lens[seq]:
             return Status.INVALID_ARG
         b = self.tables[seq][pos // self.B]
-        if self.ref[b] > 1:
+        if self.ref[b] > 1 or b in self.key_of:
             return Status.SHARED_BLOCK
         return b, pos % self.B
+
+    # ---------------------------------------------------------- prefix cache
+    def _prefix(self, tokens, i: int) -> tuple:
+        """The token prefix that logical block i ends: tokens[0 : (i+1)*B]."""
+        return tuple(int(t) for t in tokens[: (i + 1) * self.B])
+
+    def register(self, seq: int, tokens) -> Status:
+        """Register the full blocks of `seq` that `tokens` (its first n tokens,
+        n <= length, KV already written) covers, each under its prefix."""
+        if not 0 <= seq < self.max_seqs:
+            return Status.INVALID_ARG
+        if seq not in self.tables:
+            return Status.NO_SEQ
+        n = len(tokens)
+        if n > self.lens[seq]:
+            return Status.INVALID_ARG
+        table = self.tables[seq]
+        m = n // self.B
+        for i in range(m):
+            b = table[i]
+            if b in self.key_of and self.key_of[b] != self._prefix(tokens, i):
+                return Status.INVALID_ARG
+        for i in range(m):
+            b, key = table[i], self._prefix(tokens, i)
+            if key not in self.registry and b not in self.key_of:
+                self.registry[key] = b
+                self.key_of[b] = key
+        return Status.OK
+
+    def match(self, tokens) -> int:
+        """Number of leading full blocks of `tokens` whose prefix is registered."""
+        m = 0
+        while (m + 1) * self.B <= len(tokens) and self._prefix(tokens, m) in self.registry:
+            m += 1
+        return m
+
+    def reserve_prefix(self, seq: int, tokens):
+        """Create `seq` for the prompt `tokens`, reusing its cached leading
+        blocks.  Returns (Status, number of prompt tokens whose KV is cached)."""
+        n = len(tokens)
+        if not 0 <= seq < self.max_seqs or _ceil_div(n, self.B) > self.mbps:
+            return Status.INVALID_ARG, 0
+        if seq in self.tables:
+            return Status.SEQ_EXISTS, 0
+        m = self.match(tokens)
+        hit = [self.registry[self._prefix(tokens, i)] for i in range(m)]
+        idle = sum(1 for b in hit if b in self.cached)
+        need = _ceil_div(n, self.B) - m
+        if need > len(self.free) + len(self.cached) - idle:
+            return Status.NO_BLOCKS, 0
+        for b in hit:
+            self.cached.pop(b, None)
+            self.ref[b] += 1
+        table = list(hit)
+        for _ in range(need):
+            b = self._take()
+            self.ref[b] = 1
+            table.append(b)
+        self.tables[seq] = table
+        self.lens[seq] = n
+        return Status.OK, m * self.B
 
     # ----------------------------------------------------------------- cache
     def append(self, layer: int, seqs, positions, k_bits, v_bits, act_dtype: str,
@@ -235,6 +339,10 @@ class PagedKVOracle:
     def free_list(self) -> list[int]:
         return list(self.free)
 
+    def cached_list(self) -> list[int]:
+        """Registered blocks with no reference, least recently used first."""
+        return list(self.cached)
+
     def refcounts(self) -> list[int]:
         return list(self.ref)
 
@@ -247,7 +355,10 @@ class PagedKVOracle:
         * a block is on the free list iff nothing references it ("Managing
           the KV Cache", Block Tables and Sharing);
         * every block is either free or referenced, never both, never twice
-          on the free list; total references = total table entries.
+          on the free list; total references = total table entries;
+        * a block that nothing references is either free or cached, and a
+          cached block is registered; registry and key_of are inverse maps,
+          and a registered prefix is a whole number of blocks long.
         """
         counted = [0] * self.num_blocks
         for seq, table in self.tables.items():
@@ -259,5 +370,11 @@ class PagedKVOracle:
         assert counted == self.ref
         free = list(self.free)
         assert len(set(free)) == len(free)
-        assert set(free) == {b for b in range(self.num_blocks) if self.ref[b] == 0}
-        assert len(free) + sum(1 for r in self.ref if r > 0) == self.num_blocks
+        idle = set(free) | set(self.cached)
+        assert not set(free) & set(self.cached)
+        assert idle == {b for b in range(self.num_blocks) if self.ref[b] == 0}
+        assert len(free) + len(self.cached) + sum(1 for r in self.ref if r > 0) == self.num_blocks
+        assert all(b in self.key_of for b in self.cached)
+        assert not set(free) & set(self.key_of)
+        assert {v: k for k, v in self.registry.items()} == self.key_of
+        assert all(len(k) % self.B == 0 and len(k) > 0 for k in self.registry)

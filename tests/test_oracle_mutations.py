@@ -17,6 +17,7 @@ from oracle import fp8, paged, sizing
 import test_oracle_attention as att
 import test_oracle_fp8 as tf8
 import test_oracle_pool as pool
+import test_oracle_prefix as pfx
 import test_oracle_sizing as tsz
 
 
@@ -54,14 +55,34 @@ MUTANTS = [
      lambda: att.test_matches_scalar_brute_force(1)),
     (paged.PagedKVOracle, "reserve", "cow = new_len > cur and cur % self.B != 0 and self.ref[table[-1]] > 1",
      "cow = False", lambda: pool.test_parallel_sampling_cow_seven_copies_one_in_place()),
-    (paged.PagedKVOracle, "reserve", "if int(cow) + grow > len(self.free):", "if grow > len(self.free):",
+    (paged.PagedKVOracle, "reserve", "if int(cow) + grow > len(self.free) + len(self.cached):",
+     "if grow > len(self.free) + len(self.cached):",
      lambda: pool.test_cow_and_growth_need_is_checked_before_any_change()),
     (paged.PagedKVOracle, "release", "self.free.append(b)", "self.free.appendleft(b)",
      lambda: pool.test_release_returns_blocks_in_logical_order_once_unreferenced()),
-    (paged.PagedKVOracle, "slot", "if self.ref[b] > 1:", "if self.ref[b] > 2:",
+    (paged.PagedKVOracle, "slot", "if self.ref[b] > 1 or", "if self.ref[b] > 2 or",
      lambda: pool.test_invalid_calls()),
     (paged.PagedKVOracle, "append", "self.k[layer][b, :, o, :] = k_bits[t]", "self.k[layer][b, :, o - 1, :] = k_bits[t]",
      lambda: pool.test_append_writes_the_slot_and_nothing_else()),
+    # block-granular prefix cache
+    (paged.PagedKVOracle, "_prefix", "tokens[: (i + 1) * self.B]", "tokens[i * self.B : (i + 1) * self.B]",
+     lambda: pfx.test_conversations_under_pool_pressure_keep_exact_contents(0)),
+    (paged.PagedKVOracle, "_take", "popitem(last=False)", "popitem(last=True)",
+     lambda: pfx.test_lru_trace_by_hand()),
+    (paged.PagedKVOracle, "_take", "del self.registry[self.key_of.pop(b)]", "self.key_of.pop(b)",
+     lambda: pfx.test_conversations_under_pool_pressure_keep_exact_contents(0)),
+    (paged.PagedKVOracle, "release", "for b in reversed(self.tables[seq]):", "for b in self.tables[seq]:",
+     lambda: pfx.test_lru_trace_by_hand()),
+    (paged.PagedKVOracle, "release", "if self.ref[b] == 0 and b not in self.key_of:", "if self.ref[b] == 0:",
+     lambda: pfx.test_lru_trace_by_hand()),
+    (paged.PagedKVOracle, "slot", "or b in self.key_of", "or False",
+     lambda: pfx.test_registered_blocks_are_immutable_and_first_registration_wins()),
+    (paged.PagedKVOracle, "register", "if key not in self.registry and b not in self.key_of:",
+     "if b not in self.key_of:",
+     lambda: pfx.test_registered_blocks_are_immutable_and_first_registration_wins()),
+    (paged.PagedKVOracle, "reserve_prefix", "if need > len(self.free) + len(self.cached) - idle:",
+     "if need > len(self.free) + len(self.cached):",
+     lambda: pfx.test_reusing_every_idle_block_and_needing_one_more_fails_cleanly()),
 ]
 
 
@@ -87,7 +108,7 @@ def test_planted_mistake_is_caught(case, monkeypatch, golden_dir):
             _sizing_pins(golden_dir)
         return
     # an assertion, or the mutant crashing on a state the real code never reaches
-    with pytest.raises((AssertionError, IndexError)):
+    with pytest.raises((AssertionError, IndexError, KeyError)):
         pin()
 
 
