@@ -14,7 +14,8 @@
  *   [MKV] "Managing the KV Cache": Reproduce Bytes per Token, Internal
  *         Fragmentation, Block Tables and Sharing, Quantized KV, Answer Key;
  *   [PAS] "kv-cache-pagedattention-serving": PagedAttention: virtual memory
- *         for GPUs; The bonus: sharing via copy-on-write.
+ *         for GPUs; The bonus: sharing via copy-on-write; Beyond paging:
+ *         radix trees and continuous batching (block-granular prefix cache).
  *
  * Conventions for every call:
  *   - Every call returns a pa_status.  Out-parameters are written only when
@@ -127,7 +128,8 @@ void pa_pool_destroy(pa_pool *pool);
 /* Reserve slots so sequence `seq` holds `new_len` tokens, creating it if
  * it does not exist.  Blocks are taken from the head of the free list only
  * when the sequence crosses a block boundary ([KVC] paging paragraph; [MKV]
- * Answer Key item 2).  If the sequence's partly filled tail block is shared
+ * Answer Key item 2); with the free list empty, the least recently used
+ * cached block is evicted and taken instead (prefix cache, below).  If the sequence's partly filled tail block is shared
  * with other sequences and the reservation grows the sequence, the tail is
  * first copied to a fresh block (copy-on-write, [MKV] Block Tables and
  * Sharing; [PAS] The bonus: sharing via copy-on-write); the copy covers the
@@ -232,8 +234,56 @@ pa_status pa_decode_attention_noalloc(const pa_pool_desc *desc, int32_t layer, i
 
 /* Drop `seq`: every block's reference count falls by one, and blocks that
  * reach zero go to the tail of the free list in logical-block order ([MKV]
- * Block Tables and Sharing).  Errors: PA_ERR_INVALID_ARG, PA_ERR_NO_SEQ. */
+ * Block Tables and Sharing) -- registered ones (prefix cache, below) to the
+ * recently used end of the cached list instead, in reverse logical order.
+ * Errors: PA_ERR_INVALID_ARG, PA_ERR_NO_SEQ. */
 pa_status pa_free(pa_pool *pool, int32_t seq);
+
+/* ---- block-granular prefix cache ([PAS] Beyond paging: radix trees and
+ * continuous batching; [MKV] Block Tables and Sharing, Answer Key item 4) ----
+ *
+ * A full block whose KV the caller has written, in every layer, may be
+ * registered under the token prefix it ends: every token from the start of
+ * its sequence to its last slot (a token's KV depends on all tokens before
+ * it).  A new prompt then reuses, from its first block on, each block whose
+ * whole prefix is registered, and stops at the first one that is not; reuse
+ * is whole blocks only (a 103-token prompt reuses at most 96 tokens with
+ * 16-token blocks).  Registered blocks are reference counted like any other.
+ * Once nothing references one it is kept, contents intact, on a least-
+ * recently-used list (pa_get_cached_blocks) instead of the free list, and it
+ * is evicted -- unregistered and handed out again -- only when a block is
+ * needed and the free list is empty.  A registered block is immutable:
+ * pa_append_kv and pa_decode_attention_append refuse to write into it
+ * (PA_ERR_SHARED_BLOCK).  The first registration of a prefix wins.  Tokens
+ * are opaque int32 ids compared exactly; all of this is host work. */
+
+/* Register the full blocks of `seq` that cover tokens[0, n_tokens), the
+ * sequence's first n_tokens tokens (n_tokens <= its length; `tokens` is a
+ * host array, may be NULL when n_tokens == 0).  A block whose prefix is
+ * already registered under another block stays unregistered.
+ * Errors: PA_ERR_INVALID_ARG (n_tokens negative or beyond the length; a block
+ * already registered under a different prefix -- nothing is registered
+ * then), PA_ERR_NO_SEQ. */
+pa_status pa_prefix_register(pa_pool *pool, int32_t seq, int32_t n_tokens, const int32_t *tokens);
+
+/* *n_cached = how many leading tokens of the prompt tokens[0, n_tokens) have
+ * their KV in registered blocks (a multiple of block_size).  Changes nothing.
+ * Errors: PA_ERR_INVALID_ARG. */
+pa_status pa_prefix_match(const pa_pool *pool, int32_t n_tokens, const int32_t *tokens,
+                          int32_t *n_cached);
+
+/* Create `seq` with length n_tokens for the prompt tokens[0, n_tokens): its
+ * leading blocks whose prefix is registered are shared (reference count + 1;
+ * an idle one leaves the cached list), the rest are taken from the free list
+ * and then by evicting cached blocks.  *n_cached = prompt tokens whose KV the
+ * shared blocks already hold; the caller appends positions n_cached ..
+ * n_tokens - 1 and may then register the prompt.  No device work: the new
+ * table reaches the device with the next kernel launch on the pool.
+ * Errors: PA_ERR_INVALID_ARG (seq out of range, n_tokens negative or beyond
+ * max_blocks_per_seq * block_size), PA_ERR_SEQ_EXISTS, PA_ERR_NO_BLOCKS
+ * (checked before any change). */
+pa_status pa_alloc_blocks_prefix(pa_pool *pool, int32_t seq, int32_t n_tokens,
+                                 const int32_t *tokens, int32_t *n_cached);
 
 /* ---- introspection (host state; for tests and schedulers) ---- */
 
@@ -245,6 +295,9 @@ pa_status pa_get_seq(pa_pool *pool, int32_t seq, int32_t *len, int32_t *table, i
 pa_status pa_get_refcounts(pa_pool *pool, int32_t *out, int32_t cap);
 /* Free list from head to tail: `out` receives min(cap, *n) entries. */
 pa_status pa_get_free_list(pa_pool *pool, int32_t *out, int32_t cap, int32_t *n);
+/* Cached blocks (registered, unreferenced), least recently used first:
+ * `out` receives min(cap, *n) entries. */
+pa_status pa_get_cached_blocks(pa_pool *pool, int32_t *out, int32_t cap, int32_t *n);
 /* Every copy-on-write made so far as (src, dst) pairs: `pairs` receives
  * min(cap, *n) pairs (2 ints each). */
 pa_status pa_get_cow_log(pa_pool *pool, int32_t *pairs, int32_t cap, int32_t *n);

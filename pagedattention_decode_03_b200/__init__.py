@@ -28,6 +28,7 @@ from .binding import (  # noqa: F401
     lib,
     pa_alloc_blocks,
     pa_alloc_blocks_n,
+    pa_alloc_blocks_prefix,
     pa_append_kv,
     pa_check_device_errors,
     pa_debug_fail_after,
@@ -36,11 +37,14 @@ from .binding import (  # noqa: F401
     pa_decode_attention_noalloc,
     pa_fork_cow,
     pa_free,
+    pa_get_cached_blocks,
     pa_get_cow_log,
     pa_get_free_list,
     pa_get_refcounts,
     pa_last_decode_plan,
     pa_plan_siblings,
+    pa_prefix_match,
+    pa_prefix_register,
     pa_get_seq,
     pa_last_error,
     pa_launch_count,

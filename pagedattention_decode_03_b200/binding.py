@@ -39,7 +39,8 @@ EXPORTS = (
     "pa_get_seq", "pa_get_refcounts", "pa_get_free_list", "pa_get_cow_log", "pa_launch_count",
     "pa_check_device_errors", "pa_debug_fail_after", "pa_last_error", "pa_status_string",
     "pa_decode_attention_noalloc", "pa_last_decode_plan", "pa_decode_attention_append",
-    "pa_plan_siblings",
+    "pa_plan_siblings", "pa_prefix_register", "pa_prefix_match", "pa_alloc_blocks_prefix",
+    "pa_get_cached_blocks",
 )
 
 
@@ -103,6 +104,10 @@ def lib() -> ctypes.CDLL:
         L.pa_decode_attention_noalloc.argtypes = [ctypes.POINTER(pa_pool_desc), i32, i32, vp, _i32p,
                                                   i32, vp, vp, ctypes.c_float, vp]
         L.pa_free.argtypes = [vp, i32]
+        L.pa_prefix_register.argtypes = [vp, i32, i32, _i32p]
+        L.pa_prefix_match.argtypes = [vp, i32, _i32p, _i32p]
+        L.pa_alloc_blocks_prefix.argtypes = [vp, i32, i32, _i32p, _i32p]
+        L.pa_get_cached_blocks.argtypes = [vp, _i32p, i32, _i32p]
         L.pa_get_seq.argtypes = [vp, i32, _i32p, _i32p, i32, _i32p]
         L.pa_get_refcounts.argtypes = [vp, _i32p, i32]
         L.pa_get_free_list.argtypes = [vp, _i32p, i32, _i32p]
@@ -280,6 +285,29 @@ def pa_free(pool: Pool, seq: int) -> None:
     _check(lib().pa_free(pool.handle, seq), "pa_free")
 
 
+def pa_prefix_register(pool: Pool, seq: int, tokens) -> None:
+    """Register the full blocks of `seq` that its first len(tokens) tokens cover."""
+    t = _i32(tokens)
+    _check(lib().pa_prefix_register(pool.handle, seq, len(t), _ptr(t)), "pa_prefix_register")
+
+
+def pa_prefix_match(pool: Pool, tokens) -> int:
+    """Leading prompt tokens whose KV registered blocks hold."""
+    t = _i32(tokens)
+    c = ctypes.c_int32()
+    _check(lib().pa_prefix_match(pool.handle, len(t), _ptr(t), ctypes.byref(c)), "pa_prefix_match")
+    return c.value
+
+
+def pa_alloc_blocks_prefix(pool: Pool, seq: int, tokens) -> int:
+    """Create `seq` for the prompt `tokens`; returns the cached prompt tokens."""
+    t = _i32(tokens)
+    c = ctypes.c_int32()
+    _check(lib().pa_alloc_blocks_prefix(pool.handle, seq, len(t), _ptr(t), ctypes.byref(c)),
+           "pa_alloc_blocks_prefix")
+    return c.value
+
+
 def _dev_tensor(t, name, rows, heads, act):
     import torch
     want = torch.bfloat16 if act == "bf16" else torch.float16
@@ -373,6 +401,14 @@ def pa_get_free_list(pool: Pool):
     out = np.zeros(pool.num_blocks, np.int32)
     _check(lib().pa_get_free_list(pool.handle, _ptr(out), pool.num_blocks, ctypes.byref(n)),
            "pa_get_free_list")
+    return out[: n.value].tolist()
+
+
+def pa_get_cached_blocks(pool: Pool):
+    n = ctypes.c_int32()
+    out = np.zeros(pool.num_blocks, np.int32)
+    _check(lib().pa_get_cached_blocks(pool.handle, _ptr(out), pool.num_blocks, ctypes.byref(n)),
+           "pa_get_cached_blocks")
     return out[: n.value].tolist()
 
 

@@ -458,6 +458,36 @@ pa_status pa_free(pa_pool* p, int32_t seq) {
   return bm_status(p->bm->release(seq), "pa_free");
 }
 
+pa_status pa_prefix_register(pa_pool* p, int32_t seq, int32_t n_tokens, const int32_t* tokens) {
+  g_last_error.clear();
+  if (!p || n_tokens < 0 || (n_tokens > 0 && !tokens)) return fail(PA_ERR_INVALID_ARG, "null argument");
+  pa_status st = seq_arg(p, seq);
+  if (st != PA_OK) return st;
+  return bm_status(p->bm->register_prefix(seq, n_tokens, tokens), "pa_prefix_register");
+}
+
+pa_status pa_prefix_match(const pa_pool* p, int32_t n_tokens, const int32_t* tokens,
+                          int32_t* n_cached) {
+  g_last_error.clear();
+  if (!p || !n_cached || n_tokens < 0 || (n_tokens > 0 && !tokens))
+    return fail(PA_ERR_INVALID_ARG, "null argument");
+  *n_cached = p->bm->match_prefix(n_tokens, tokens, nullptr) * p->d.block_size;
+  return PA_OK;
+}
+
+pa_status pa_alloc_blocks_prefix(pa_pool* p, int32_t seq, int32_t n_tokens, const int32_t* tokens,
+                                 int32_t* n_cached) {
+  g_last_error.clear();
+  if (!p || !n_cached || n_tokens < 0 || (n_tokens > 0 && !tokens))
+    return fail(PA_ERR_INVALID_ARG, "null argument");
+  pa_status st = seq_arg(p, seq);
+  if (st != PA_OK) return st;
+  int32_t c = 0;
+  st = bm_status(p->bm->reserve_prefix(seq, n_tokens, tokens, &c), "pa_alloc_blocks_prefix");
+  if (st == PA_OK) *n_cached = c;
+  return st;
+}
+
 pa_status pa_append_kv(pa_pool* p, int32_t layer, int32_t T, const int32_t* seqs,
                        const int32_t* positions, const void* k_new, const void* v_new,
                        void* stream) {
@@ -712,6 +742,17 @@ pa_status pa_get_free_list(pa_pool* p, int32_t* out, int32_t cap, int32_t* n) {
   const int32_t m = std::min<int32_t>(cap, static_cast<int32_t>(fl.size()));
   if (m > 0) std::memcpy(out, fl.data(), sizeof(int32_t) * m);
   *n = static_cast<int32_t>(fl.size());
+  return PA_OK;
+}
+
+pa_status pa_get_cached_blocks(pa_pool* p, int32_t* out, int32_t cap, int32_t* n) {
+  g_last_error.clear();
+  if (!p || !n || (cap > 0 && !out)) return fail(PA_ERR_INVALID_ARG, "null argument");
+  std::vector<int32_t> cl;
+  p->bm->cached_list(&cl);
+  const int32_t m = std::min<int32_t>(cap, static_cast<int32_t>(cl.size()));
+  if (m > 0) std::memcpy(out, cl.data(), sizeof(int32_t) * m);
+  *n = static_cast<int32_t>(cl.size());
   return PA_OK;
 }
 

@@ -2,6 +2,7 @@
 #include "block_manager.h"
 
 #include <algorithm>
+#include <cstring>
 
 namespace pa {
 
@@ -33,7 +34,8 @@ void MirrorDeltas::consume(size_t n) {
 BlockManager::BlockManager(int32_t num_blocks, int32_t block_size, int32_t max_seqs,
                            int32_t max_blocks_per_seq, const int32_t* free_order)
     : num_blocks_(num_blocks), block_size_(block_size), max_seqs_(max_seqs),
-      mbps_(max_blocks_per_seq), ring_(num_blocks), ref_(num_blocks, 0), seqs_(max_seqs) {
+      mbps_(max_blocks_per_seq), ring_(num_blocks), ref_(num_blocks, 0), seqs_(max_seqs),
+      block_node_(num_blocks, -1), lru_prev_(num_blocks, -2), lru_next_(num_blocks, -2) {
   for (int32_t b = 0; b < num_blocks; ++b) ring_[b] = free_order ? free_order[b] : b;
   free_count_ = num_blocks;
   deltas_.reset(static_cast<int64_t>(max_seqs) * max_blocks_per_seq + max_seqs);
@@ -51,6 +53,107 @@ void BlockManager::push_free(int32_t b) {
   if (tail >= num_blocks_) tail -= num_blocks_;
   ring_[tail] = b;
   ++free_count_;
+}
+
+int32_t BlockManager::take_block() {
+  if (free_count_ > 0) return pop_free();
+  const int32_t b = lru_head_;
+  lru_remove(b);
+  unregister(b);
+  return b;
+}
+
+void BlockManager::lru_push_back(int32_t b) {
+  lru_prev_[b] = lru_tail_;
+  lru_next_[b] = -1;
+  if (lru_tail_ >= 0) lru_next_[lru_tail_] = b; else lru_head_ = b;
+  lru_tail_ = b;
+  ++lru_count_;
+}
+
+void BlockManager::lru_remove(int32_t b) {
+  const int32_t p = lru_prev_[b], n = lru_next_[b];
+  if (p >= 0) lru_next_[p] = n; else lru_head_ = n;
+  if (n >= 0) lru_prev_[n] = p; else lru_tail_ = p;
+  lru_prev_[b] = lru_next_[b] = -2;
+  --lru_count_;
+}
+
+uint64_t BlockManager::node_key(int32_t parent, const int32_t* toks) const {
+  // FNV-1a over the parent id and the tokens, then the MurmurHash3 64-bit
+  // finaliser to spread the bits over the buckets.
+  uint64_t h = 0xcbf29ce484222325ull;
+  auto mix = [&h](uint32_t w) {
+    for (int k = 0; k < 4; ++k) {
+      h ^= (w >> (8 * k)) & 0xffu;
+      h *= 0x100000001b3ull;
+    }
+  };
+  mix(static_cast<uint32_t>(parent));
+  for (int32_t i = 0; i < block_size_; ++i) mix(static_cast<uint32_t>(toks[i]));
+  h ^= h >> 33;
+  h *= 0xff51afd7ed558ccdull;
+  h ^= h >> 33;
+  h *= 0xc4ceb9fe1a85ec53ull;
+  h ^= h >> 33;
+  return h;
+}
+
+int32_t BlockManager::find_child(int32_t parent, const int32_t* toks) const {
+  const auto range = index_.equal_range(node_key(parent, toks));
+  for (auto it = range.first; it != range.second; ++it) {
+    const int32_t c = it->second;
+    if (nodes_[c].parent == parent &&
+        std::memcmp(&node_tokens_[static_cast<size_t>(c) * block_size_], toks,
+                    sizeof(int32_t) * block_size_) == 0)
+      return c;
+  }
+  return -1;
+}
+
+int32_t BlockManager::add_child(int32_t parent, const int32_t* toks) {
+  int32_t c;
+  if (!spare_nodes_.empty()) {
+    c = spare_nodes_.back();
+    spare_nodes_.pop_back();
+  } else {
+    c = static_cast<int32_t>(nodes_.size());
+    nodes_.push_back({});
+    node_tokens_.resize(nodes_.size() * static_cast<size_t>(block_size_));
+  }
+  const uint64_t key = node_key(parent, toks);
+  nodes_[c] = {parent, -1, 0, key};
+  std::memcpy(&node_tokens_[static_cast<size_t>(c) * block_size_], toks,
+              sizeof(int32_t) * block_size_);
+  index_.emplace(key, c);
+  if (parent >= 0) ++nodes_[parent].children;
+  return c;
+}
+
+// Drop nodes that hold no block and lead to none, walking towards the root.
+// A node is only dropped once no child names it as parent, so a reused node
+// id never matches a stale key.
+void BlockManager::prune(int32_t node) {
+  while (node >= 0 && nodes_[node].block < 0 && nodes_[node].children == 0) {
+    const auto range = index_.equal_range(nodes_[node].key);
+    for (auto it = range.first; it != range.second; ++it) {
+      if (it->second == node) {
+        index_.erase(it);
+        break;
+      }
+    }
+    const int32_t parent = nodes_[node].parent;
+    spare_nodes_.push_back(node);
+    if (parent >= 0) --nodes_[parent].children;
+    node = parent;
+  }
+}
+
+void BlockManager::unregister(int32_t block) {
+  const int32_t node = block_node_[block];
+  block_node_[block] = -1;
+  nodes_[node].block = -1;
+  prune(node);
 }
 
 void BlockManager::record_entry(int32_t seq, int32_t j, int32_t block) {
@@ -73,7 +176,7 @@ Status BlockManager::reserve(int32_t seq, int32_t new_len, std::vector<CowPair>*
   const bool cow = new_len > cur && (cur % block_size_) != 0 && ref_[s.table.back()] > 1;
   const int64_t grow = want_blocks - have;
   const int64_t need = (cow ? 1 : 0) + grow;
-  if (need > free_count_) return kNoBlocks;
+  if (need > static_cast<int64_t>(free_count_) + lru_count_) return kNoBlocks;
   if (fail_after_ >= 0 && need > fail_after_) return kNoBlocks;
 
   if (!s.active) {
@@ -84,7 +187,7 @@ Status BlockManager::reserve(int32_t seq, int32_t new_len, std::vector<CowPair>*
   }
   if (cow) {
     const int32_t src = s.table.back();
-    const int32_t dst = pop_free();
+    const int32_t dst = take_block();
     --ref_[src];
     ref_[dst] = 1;
     s.table.back() = dst;
@@ -92,7 +195,7 @@ Status BlockManager::reserve(int32_t seq, int32_t new_len, std::vector<CowPair>*
     cows->push_back({src, dst});
   }
   for (int64_t k = 0; k < grow; ++k) {
-    const int32_t b = pop_free();
+    const int32_t b = take_block();
     ref_[b] = 1;
     s.table.push_back(b);
     record_entry(seq, static_cast<int32_t>(s.table.size()) - 1, b);
@@ -125,7 +228,10 @@ Status BlockManager::release(int32_t seq) {
   Seq& s = seqs_[seq];
   if (!s.active) return kNoSeq;
   for (int32_t b : s.table) {
-    if (--ref_[b] == 0) push_free(b);
+    if (--ref_[b] == 0 && block_node_[b] < 0) push_free(b);
+  }
+  for (auto it = s.table.rbegin(); it != s.table.rend(); ++it) {
+    if (ref_[*it] == 0 && block_node_[*it] >= 0) lru_push_back(*it);
   }
   s.active = false;
   s.len = 0;
@@ -140,9 +246,96 @@ Status BlockManager::slot(int32_t seq, int32_t pos, int64_t* slot_out) const {
   if (!s.active) return kNoSeq;
   if (pos < 0 || pos >= s.len) return kInvalidArg;
   const int32_t b = s.table[pos / block_size_];
-  if (ref_[b] > 1) return kSharedBlock;
+  if (ref_[b] > 1 || block_node_[b] >= 0) return kSharedBlock;
   *slot_out = static_cast<int64_t>(b) * block_size_ + pos % block_size_;
   return kOk;
+}
+
+Status BlockManager::register_prefix(int32_t seq, int32_t n, const int32_t* tokens) {
+  if (seq < 0 || seq >= max_seqs_ || n < 0 || (n > 0 && tokens == nullptr)) return kInvalidArg;
+  Seq& s = seqs_[seq];
+  if (!s.active) return kNoSeq;
+  if (n > s.len) return kInvalidArg;
+  const int32_t m = n / block_size_;
+  // validate: a block registered already must hold this very prefix
+  int32_t node = -1;
+  bool path = true;
+  for (int32_t i = 0; i < m; ++i) {
+    const int32_t* toks = tokens + static_cast<int64_t>(i) * block_size_;
+    node = path ? find_child(node, toks) : -1;
+    path = node >= 0;
+    const int32_t bn = block_node_[s.table[i]];
+    if (bn >= 0 && bn != node) return kInvalidArg;
+  }
+  node = -1;
+  for (int32_t i = 0; i < m; ++i) {
+    const int32_t* toks = tokens + static_cast<int64_t>(i) * block_size_;
+    int32_t c = find_child(node, toks);
+    if (c < 0) c = add_child(node, toks);
+    const int32_t b = s.table[i];
+    if (nodes_[c].block < 0 && block_node_[b] < 0) {
+      nodes_[c].block = b;
+      block_node_[b] = c;
+    }
+    node = c;
+  }
+  return kOk;
+}
+
+int32_t BlockManager::match_prefix(int32_t n, const int32_t* tokens,
+                                   std::vector<int32_t>* blocks) const {
+  if (blocks) blocks->clear();
+  int32_t node = -1, m = 0;
+  for (; (static_cast<int64_t>(m) + 1) * block_size_ <= n; ++m) {
+    const int32_t c = find_child(node, tokens + static_cast<int64_t>(m) * block_size_);
+    if (c < 0 || nodes_[c].block < 0) break;
+    if (blocks) blocks->push_back(nodes_[c].block);
+    node = c;
+  }
+  return m;
+}
+
+Status BlockManager::reserve_prefix(int32_t seq, int32_t n, const int32_t* tokens,
+                                    int32_t* n_cached) {
+  if (seq < 0 || seq >= max_seqs_ || n < 0 || (n > 0 && tokens == nullptr)) return kInvalidArg;
+  const int64_t want_blocks = (static_cast<int64_t>(n) + block_size_ - 1) / block_size_;
+  if (want_blocks > mbps_) return kInvalidArg;
+  Seq& s = seqs_[seq];
+  if (s.active) return kSeqExists;
+  std::vector<int32_t> hit;
+  const int32_t m = match_prefix(n, tokens, &hit);
+  int64_t idle = 0;
+  for (int32_t b : hit) idle += ref_[b] == 0 ? 1 : 0;
+  const int64_t need = want_blocks - m;
+  if (need > static_cast<int64_t>(free_count_) + lru_count_ - idle) return kNoBlocks;
+  if (fail_after_ >= 0 && need > fail_after_) return kNoBlocks;
+
+  s.active = true;
+  s.table.clear();
+  s.table.reserve(static_cast<size_t>(std::min<int64_t>(mbps_, want_blocks + 64)));
+  for (int32_t b : hit) {
+    if (ref_[b] == 0) lru_remove(b);
+    ++ref_[b];
+    s.table.push_back(b);
+    record_entry(seq, static_cast<int32_t>(s.table.size()) - 1, b);
+  }
+  for (int64_t k = 0; k < need; ++k) {
+    const int32_t b = take_block();
+    ref_[b] = 1;
+    s.table.push_back(b);
+    record_entry(seq, static_cast<int32_t>(s.table.size()) - 1, b);
+  }
+  if (fail_after_ >= 0) fail_after_ -= need;
+  s.len = n;
+  record_len(seq, n);
+  *n_cached = m * block_size_;
+  return kOk;
+}
+
+void BlockManager::cached_list(std::vector<int32_t>* out) const {
+  out->clear();
+  out->reserve(lru_count_);
+  for (int32_t b = lru_head_; b >= 0; b = lru_next_[b]) out->push_back(b);
 }
 
 void BlockManager::free_list(std::vector<int32_t>* out) const {

@@ -13,12 +13,30 @@
 // that needs a copy-on-write block and new blocks takes the copy-on-write
 // block first; the need is checked before any change.
 //
+// Block-granular prefix cache (kv-cache-pagedattention-serving, Beyond
+// paging: radix trees and continuous batching; "Managing the KV Cache",
+// Block Tables and Sharing): a full block whose KV is written may be
+// registered under the token prefix it ends (every token from the sequence
+// start to its last slot).  A new prompt reuses, from its first block on,
+// each block whose whole prefix is registered, and stops at the first miss.
+// The index is a trie with one node per distinct whole-block prefix, found by
+// (parent node, the block's own tokens) and compared exactly, so no hash
+// collision can hand out a wrong block.  Registered blocks that nothing
+// references stay on a least-recently-used list with their contents and are
+// evicted only when a block is needed and the free list is empty.  Where the
+// pages are silent: a registered block is immutable (a write into it is
+// refused like a write into a shared block); the first registration of a
+// prefix wins; a release adds its registered blocks to the recently-used end
+// in reverse logical order, so a longer prefix is evicted before the shorter
+// one it extends.
+//
 // Every change that the device must see (a block-table entry, a sequence
 // length) is recorded in a MirrorDeltas list, which the API layer ships to
 // the device copy of the tables with the next kernel launch.
 #pragma once
 
 #include <cstdint>
+#include <unordered_map>
 #include <vector>
 
 namespace pa {
@@ -69,6 +87,22 @@ class BlockManager {
   // Flat slot id (block * block_size + offset) of token `pos` of `seq`.
   Status slot(int32_t seq, int32_t pos, int64_t* slot_out) const;
 
+  // Prefix cache.  `tokens` holds the first `n` tokens of the sequence.
+  // register_prefix: registers the full blocks of `seq` covering tokens[0, n),
+  // n <= length; fails (nothing registered) if one of them is already
+  // registered under another prefix.
+  Status register_prefix(int32_t seq, int32_t n, const int32_t* tokens);
+  // Leading full blocks of tokens[0, n) whose prefix is registered; their
+  // block ids go to `blocks` if given.
+  int32_t match_prefix(int32_t n, const int32_t* tokens, std::vector<int32_t>* blocks) const;
+  // Create `seq` for the prompt tokens[0, n), reusing its cached leading
+  // blocks; *n_cached = the prompt tokens whose KV those blocks hold.
+  Status reserve_prefix(int32_t seq, int32_t n, const int32_t* tokens, int32_t* n_cached);
+  int32_t cached_count() const { return lru_count_; }
+  // Registered blocks with no reference, least recently used first.
+  void cached_list(std::vector<int32_t>* out) const;
+  bool registered(int32_t block) const { return block_node_[block] >= 0; }
+
   bool active(int32_t seq) const { return seq >= 0 && seq < max_seqs_ && seqs_[seq].active; }
   int32_t len(int32_t seq) const { return seqs_[seq].len; }
   const std::vector<int32_t>& table(int32_t seq) const { return seqs_[seq].table; }
@@ -90,8 +124,24 @@ class BlockManager {
     int32_t len = 0;
     std::vector<int32_t> table;
   };
+  // One distinct whole-block token prefix: its last block's tokens live at
+  // node_tokens_[id * block_size].
+  struct Node {
+    int32_t parent;    // node of the prefix one block shorter, -1 at depth 1
+    int32_t block;     // registered block holding this prefix's last block, or -1
+    int32_t children;  // nodes whose parent is this one
+    uint64_t key;      // hash of (parent, tokens), the index key
+  };
   int32_t pop_free();
   void push_free(int32_t b);
+  int32_t take_block();  // free head, else evict the least recently used cached block
+  uint64_t node_key(int32_t parent, const int32_t* toks) const;
+  int32_t find_child(int32_t parent, const int32_t* toks) const;
+  int32_t add_child(int32_t parent, const int32_t* toks);
+  void prune(int32_t node);
+  void unregister(int32_t block);
+  void lru_push_back(int32_t b);
+  void lru_remove(int32_t b);
   void record_entry(int32_t seq, int32_t j, int32_t block);
   void record_len(int32_t seq, int32_t len);
 
@@ -102,6 +152,13 @@ class BlockManager {
   std::vector<Seq> seqs_;
   int64_t fail_after_ = -1;  // remaining allocations before injected failure
   MirrorDeltas deltas_;
+
+  std::vector<Node> nodes_;
+  std::vector<int32_t> node_tokens_, spare_nodes_;
+  std::unordered_multimap<uint64_t, int32_t> index_;  // key -> node
+  std::vector<int32_t> block_node_;                   // block -> node, or -1
+  std::vector<int32_t> lru_prev_, lru_next_;          // -2: not on the list
+  int32_t lru_head_ = -1, lru_tail_ = -1, lru_count_ = 0;
 };
 
 }  // namespace pa

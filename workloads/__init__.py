@@ -17,6 +17,7 @@ from .gen import (  # noqa: F401
     fp8_scales,
     normal_bits,
     prefill_kv_bits,
+    prefix_kv_bits,
     rng,
     step_kv_bits,
     step_q_bits,

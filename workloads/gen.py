@@ -10,6 +10,7 @@ and returned as raw uint16 bit patterns.
 from __future__ import annotations
 
 import enum
+import hashlib
 
 import numpy as np
 import torch
@@ -26,6 +27,7 @@ class Purpose(enum.IntEnum):
     K_NEW = 5
     V_NEW = 6
     MISC = 7
+    PREFIX_KV = 8
 
 
 def rng(seed: int, cfg: int, purpose: int, *extra: int) -> np.random.Generator:
@@ -69,6 +71,26 @@ def step_kv_bits(w, step: int, layer: int):
     shape = (len(w.seq_ids), w.num_kv_heads, w.head_dim)
     k = normal_bits(rng(w.seed, w.cfg, Purpose.K_NEW, step, layer), shape, w.act_dtype)
     v = normal_bits(rng(w.seed, w.cfg, Purpose.V_NEW, step, layer), shape, w.act_dtype)
+    return k, v
+
+
+def prefix_kv_bits(w, layer: int, tokens, lo: int, hi: int):
+    """K and V rows of positions lo..hi-1 of the token history `tokens`.
+
+    Each row is drawn from a generator seeded by the whole token prefix that
+    ends at its position, so two histories that start with the same tokens
+    get the same rows there, as a model's KV would.  Shape [hi - lo,
+    num_kv_heads, head_dim], activation dtype bits, each.
+    """
+    shape = (max(hi - lo, 0), w.num_kv_heads, w.head_dim)
+    k = np.zeros(shape, np.uint16)
+    v = np.zeros(shape, np.uint16)
+    toks = np.asarray(tokens, np.int64)
+    for t in range(lo, hi):
+        digest = hashlib.blake2b(toks[: t + 1].tobytes(), digest_size=8).digest()
+        g = rng(w.seed, w.cfg, Purpose.PREFIX_KV, layer, int.from_bytes(digest, "little"))
+        k[t - lo] = normal_bits(g, shape[1:], w.act_dtype)
+        v[t - lo] = normal_bits(g, shape[1:], w.act_dtype)
     return k, v
 
 
