@@ -29,7 +29,7 @@ class Run:
         w = workload("tiny", seed=seed)
         self.w = dataclasses.replace(w, name="prefix", num_blocks=nb, max_seqs=max_seqs,
                                      max_blocks_per_seq=mbps)
-        self.P = Pair(self.w)
+        self.P = Pair(self.w, min_partition=16)
         self.hist = {}
         self.done = []
         self.calls = 0
