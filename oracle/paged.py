@@ -61,6 +61,19 @@ Readings where the pages are silent:
 * a prompt whose every token falls in registered blocks reuses all of them
   (whether the last token is recomputed to get logits is a scheduler's
   choice, outside the pool).
+
+Swap-out / swap-in ("Managing the KV Cache", Offload and Hands-On Exercise;
+kv-cache-pagedattention-serving, Beyond paging: radix trees and continuous
+batching): a preempted sequence's KV moves to host memory and its blocks go
+back to the pool; paging it back takes fresh blocks and restores every
+cached token.  Readings where the pages are silent:
+
+* the transfer moves whole allocated blocks (the exercise asks for both the
+  useful-state and the allocated-block byte counts; a block-granular copy
+  moves the latter), every layer, K and V, as raw storage bits;
+* the host image is laid out [K, V][logical block][layer][kv_head][slot][dim];
+* swap-out releases the sequence exactly as a release does; swap-in creates
+  it again with private blocks (sharing with forks is not restored).
 """
 from __future__ import annotations
 
@@ -331,6 +344,42 @@ class PagedKVOracle:
                 p /= p.sum()
                 out[i, qh] = p @ vh
         return out
+
+    # ------------------------------------------------------------- swapping
+    def swap_bytes(self, n_tokens: int, bytes_per_element: int) -> int:
+        """Size of the host image of an n-token sequence: its allocated blocks,
+        every layer, K and V."""
+        return (2 * _ceil_div(n_tokens, self.B) * self.L * self.H * self.B * self.d
+                * bytes_per_element)
+
+    def swap_out(self, seq: int):
+        """(Status, host image, length): copy the blocks of `seq` out, then
+        release it.  The image holds the stored layers only:
+        [2][blocks][stored layers][kv_head][slot][dim] raw bits."""
+        if seq not in self.tables:
+            return (Status.NO_SEQ if 0 <= seq < self.max_seqs else Status.INVALID_ARG), None, 0
+        table, n = self.tables[seq], self.lens[seq]
+        layers = sorted(self.k)
+        image = np.stack([np.stack([np.stack([cache[layer][b] for layer in layers]) for b in table])
+                          for cache in (self.k, self.v)])
+        self.release(seq)
+        return Status.OK, image, n
+
+    def swap_in(self, seq: int, n_tokens: int, image) -> Status:
+        """Create `seq` with `n_tokens` tokens in fresh blocks and write the
+        host image (as swap_out returns it) into them."""
+        if not 0 <= seq < self.max_seqs:
+            return Status.INVALID_ARG
+        if seq in self.tables:
+            return Status.SEQ_EXISTS
+        st = self.reserve(seq, n_tokens)
+        if st != Status.OK:
+            return st
+        for j, b in enumerate(self.tables[seq]):
+            for i, layer in enumerate(sorted(self.k)):
+                self.k[layer][b] = image[0][j][i]
+                self.v[layer][b] = image[1][j][i]
+        return Status.OK
 
     # ------------------------------------------------------------ inspection
     def table(self, seq: int) -> list[int]:

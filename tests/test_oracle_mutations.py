@@ -18,6 +18,7 @@ import test_oracle_attention as att
 import test_oracle_fp8 as tf8
 import test_oracle_pool as pool
 import test_oracle_prefix as pfx
+import test_oracle_swap as swp
 import test_oracle_sizing as tsz
 
 
@@ -83,6 +84,19 @@ MUTANTS = [
     (paged.PagedKVOracle, "reserve_prefix", "if need > len(self.free) + len(self.cached) - idle:",
      "if need > len(self.free) + len(self.cached):",
      lambda: pfx.test_reusing_every_idle_block_and_needing_one_more_fails_cleanly()),
+    # swap-out / swap-in
+    (paged.PagedKVOracle, "swap_bytes", "(2 * _ceil_div(n_tokens, self.B)", "(_ceil_div(n_tokens, self.B)",
+     lambda: swp.test_swap_bytes_are_the_exercise_allocated_bytes()),
+    (paged.PagedKVOracle, "swap_out", "np.stack([np.stack([cache[layer][b] for layer in layers]) for b in table])",
+     "np.stack([np.stack([cache[layer][b] for b in table]) for layer in layers])",
+     lambda: swp.test_image_layout_holds_each_appended_row_at_its_place()),
+    (paged.PagedKVOracle, "swap_out", "self.release(seq)", "None",
+     lambda: swp.test_round_trip_restores_attention_exactly_and_frees_blocks()),
+    (paged.PagedKVOracle, "swap_in", "self.v[layer][b] = image[1][j][i]", "self.v[layer][b] = image[0][j][i]",
+     lambda: swp.test_round_trip_restores_attention_exactly_and_frees_blocks()),
+    (paged.PagedKVOracle, "swap_in", "for j, b in enumerate(self.tables[seq]):",
+     "for j, b in enumerate(reversed(self.tables[seq])):",
+     lambda: swp.test_round_trip_restores_attention_exactly_and_frees_blocks()),
 ]
 
 
