@@ -239,6 +239,46 @@ pa_status pa_decode_attention_noalloc(const pa_pool_desc *desc, int32_t layer, i
  * Errors: PA_ERR_INVALID_ARG, PA_ERR_NO_SEQ. */
 pa_status pa_free(pa_pool *pool, int32_t seq);
 
+/* ---- swap-out / swap-in ([MKV] Offload, Hands-On Exercise; [PAS] Beyond
+ * paging: radix trees and continuous batching) ----
+ *
+ * A preempted sequence's KV moves to host memory and its blocks return to the
+ * pool; paging it back takes fresh blocks and restores every cached token.
+ * The transfer moves whole allocated blocks, every layer, K and V, as stored
+ * (FP8 codes for an FP8 pool; the scales stay on the device).  Host image
+ * layout, row-major: [2 (K, then V)][ceil(len / block_size)][num_layers]
+ * [num_kv_heads][block_size][head_dim] kv_dtype elements.  The image is
+ * caller-owned host memory: pinned (cudaHostAlloc / cudaHostRegister) for
+ * asynchronous copies, or pageable (the copies then wait); device or managed
+ * memory is refused.  Copies are enqueued on `stream` (copy engines, no
+ * kernel) and complete in stream order; the image is complete, or the
+ * sequence's blocks hold its contents, once the stream reaches that point. */
+
+/* *bytes = size of the host image of a sequence of n_tokens tokens:
+ * 2 x ceil(n_tokens / block_size) x num_layers x num_kv_heads x block_size x
+ * head_dim x element bytes (the allocated-block bytes; the useful-state bytes
+ * are n_tokens / (ceil(n_tokens / block_size) x block_size) of that).  Works
+ * on host-only pools.  Errors: PA_ERR_INVALID_ARG. */
+pa_status pa_swap_bytes(const pa_pool *pool, int32_t n_tokens, size_t *bytes);
+
+/* Copy every block of `seq` into the host image `host` (host_bytes >=
+ * pa_swap_bytes(len)), then drop `seq` as pa_free does (shared blocks stay
+ * with their other sequences, registered ones go to the cached list).  Its
+ * length is the caller's to keep for pa_swap_in.  Later work that reuses the
+ * freed blocks must be ordered after `stream`.
+ * Errors: PA_ERR_INVALID_ARG (host-only pool, image too small or not host
+ * memory), PA_ERR_NO_SEQ, PA_ERR_CUDA (nothing released). */
+pa_status pa_swap_out(pa_pool *pool, int32_t seq, void *host, size_t host_bytes, void *stream);
+
+/* Create `seq` with n_tokens tokens in fresh blocks from the free list (then
+ * by evicting cached blocks) and copy the host image into them; the blocks
+ * are private even if the sequence shared blocks before it was swapped out.
+ * The new table reaches the device with the next kernel launch on the pool.
+ * Errors: PA_ERR_INVALID_ARG, PA_ERR_SEQ_EXISTS, PA_ERR_NO_BLOCKS (checked
+ * before any change), PA_ERR_CUDA (the sequence is dropped again). */
+pa_status pa_swap_in(pa_pool *pool, int32_t seq, int32_t n_tokens, const void *host,
+                     size_t host_bytes, void *stream);
+
 /* ---- block-granular prefix cache ([PAS] Beyond paging: radix trees and
  * continuous batching; [MKV] Block Tables and Sharing, Answer Key item 4) ----
  *

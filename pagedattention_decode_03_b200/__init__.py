@@ -51,5 +51,8 @@ from .binding import (  # noqa: F401
     pa_pool_create,
     pa_pool_destroy,
     pa_status_string,
+    pa_swap_bytes,
+    pa_swap_in,
+    pa_swap_out,
     pa_workspace_size,
 )

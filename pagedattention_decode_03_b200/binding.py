@@ -40,7 +40,7 @@ EXPORTS = (
     "pa_check_device_errors", "pa_debug_fail_after", "pa_last_error", "pa_status_string",
     "pa_decode_attention_noalloc", "pa_last_decode_plan", "pa_decode_attention_append",
     "pa_plan_siblings", "pa_prefix_register", "pa_prefix_match", "pa_alloc_blocks_prefix",
-    "pa_get_cached_blocks",
+    "pa_get_cached_blocks", "pa_swap_bytes", "pa_swap_out", "pa_swap_in",
 )
 
 
@@ -108,6 +108,9 @@ def lib() -> ctypes.CDLL:
         L.pa_prefix_match.argtypes = [vp, i32, _i32p, _i32p]
         L.pa_alloc_blocks_prefix.argtypes = [vp, i32, i32, _i32p, _i32p]
         L.pa_get_cached_blocks.argtypes = [vp, _i32p, i32, _i32p]
+        L.pa_swap_bytes.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_size_t)]
+        L.pa_swap_out.argtypes = [vp, i32, vp, ctypes.c_size_t, vp]
+        L.pa_swap_in.argtypes = [vp, i32, i32, vp, ctypes.c_size_t, vp]
         L.pa_get_seq.argtypes = [vp, i32, _i32p, _i32p, i32, _i32p]
         L.pa_get_refcounts.argtypes = [vp, _i32p, i32]
         L.pa_get_free_list.argtypes = [vp, _i32p, i32, _i32p]
@@ -402,6 +405,38 @@ def pa_get_free_list(pool: Pool):
     _check(lib().pa_get_free_list(pool.handle, _ptr(out), pool.num_blocks, ctypes.byref(n)),
            "pa_get_free_list")
     return out[: n.value].tolist()
+
+
+def pa_swap_bytes(pool: Pool, n_tokens: int) -> int:
+    """Bytes of the host image of an n_tokens-token sequence."""
+    b = ctypes.c_size_t()
+    _check(lib().pa_swap_bytes(pool.handle, n_tokens, ctypes.byref(b)), "pa_swap_bytes")
+    return b.value
+
+
+def _host_buffer(host):
+    """(address, bytes) of a contiguous CPU torch tensor or numpy array."""
+    if isinstance(host, np.ndarray):
+        if not host.flags["C_CONTIGUOUS"]:
+            raise ValueError("host image must be contiguous")
+        return host.ctypes.data, host.nbytes
+    if host.is_cuda or not host.is_contiguous():
+        raise ValueError("host image must be a contiguous CPU tensor")
+    return host.data_ptr(), host.numel() * host.element_size()
+
+
+def pa_swap_out(pool: Pool, seq: int, host, stream=None) -> None:
+    """Copy `seq`'s blocks into `host` (see pa_swap_bytes) and drop it."""
+    ptr, nbytes = _host_buffer(host)
+    _check(lib().pa_swap_out(pool.handle, seq, ctypes.c_void_p(ptr), nbytes, _stream(stream)),
+           "pa_swap_out")
+
+
+def pa_swap_in(pool: Pool, seq: int, n_tokens: int, host, stream=None) -> None:
+    """Create `seq` with n_tokens tokens in fresh blocks holding the image."""
+    ptr, nbytes = _host_buffer(host)
+    _check(lib().pa_swap_in(pool.handle, seq, n_tokens, ctypes.c_void_p(ptr), nbytes,
+                            _stream(stream)), "pa_swap_in")
 
 
 def pa_get_cached_blocks(pool: Pool):

@@ -488,6 +488,119 @@ pa_status pa_alloc_blocks_prefix(pa_pool* p, int32_t seq, int32_t n_tokens, cons
   return st;
 }
 
+namespace {
+
+// One (layer, block) tile of K or V: num_kv_heads x block_size x head_dim elements.
+size_t tile_bytes(const pa_pool_desc& d) {
+  return static_cast<size_t>(d.num_kv_heads) * d.block_size * pa::kHeadDim *
+         (d.kv_dtype == PA_FP8_E4M3 ? 1 : 2);
+}
+
+size_t swap_image_bytes(const pa_pool_desc& d, int64_t n_tokens) {
+  const int64_t blocks = (n_tokens + d.block_size - 1) / d.block_size;
+  return 2 * static_cast<size_t>(blocks) * d.num_layers * tile_bytes(d);
+}
+
+// The host image must be host memory (pinned for asynchronous copies, or
+// pageable); device or managed memory is refused.
+pa_status check_host_image(const void* host, size_t have, size_t need) {
+  if (have < need) return fail(PA_ERR_INVALID_ARG, "host image smaller than pa_swap_bytes()");
+  if (need == 0) return PA_OK;
+  if (host == nullptr) return fail(PA_ERR_INVALID_ARG, "null host image");
+  cudaPointerAttributes a{};
+  cudaError_t e = cudaPointerGetAttributes(&a, host);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "cudaPointerGetAttributes(host image)");
+  }
+  if (a.type != cudaMemoryTypeHost && a.type != cudaMemoryTypeUnregistered)
+    return fail(PA_ERR_INVALID_ARG, "the host image must be host memory");
+  return PA_OK;
+}
+
+// Copy the blocks `table` between the pool and a host image laid out
+// [K, V][logical block][layer][tile]: per (K/V, block) one 2-D copy whose rows
+// are the block's tiles in successive layers (one layer stride apart in the
+// pool, contiguous in the image).
+pa_status swap_copies(pa_pool* p, const std::vector<int32_t>& table, char* host, bool to_host,
+                      cudaStream_t s) {
+  const pa_pool_desc& d = p->d;
+  const size_t tile = tile_bytes(d);
+  const size_t layer_stride = tile * static_cast<size_t>(d.num_blocks);
+  const size_t n = table.size();
+  int max_pitch = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&max_pitch, cudaDevAttrMaxPitch, d.device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(max pitch)");
+  const cudaMemcpyKind kind = to_host ? cudaMemcpyDeviceToHost : cudaMemcpyHostToDevice;
+  for (int kv = 0; kv < 2; ++kv) {
+    char* cache = static_cast<char*>(kv ? d.v_cache : d.k_cache);
+    for (size_t j = 0; j < n; ++j) {
+      char* dev = cache + static_cast<size_t>(table[j]) * tile;
+      char* img = host + (static_cast<size_t>(kv) * n + j) * d.num_layers * tile;
+      if (layer_stride <= static_cast<size_t>(max_pitch)) {
+        e = to_host ? cudaMemcpy2DAsync(img, tile, dev, layer_stride, tile, d.num_layers, kind, s)
+                    : cudaMemcpy2DAsync(dev, layer_stride, img, tile, tile, d.num_layers, kind, s);
+      } else {
+        for (int32_t l = 0; l < d.num_layers && e == cudaSuccess; ++l) {
+          char* dl = dev + static_cast<size_t>(l) * layer_stride;
+          char* hl = img + static_cast<size_t>(l) * tile;
+          e = to_host ? cudaMemcpyAsync(hl, dl, tile, kind, s) : cudaMemcpyAsync(dl, hl, tile, kind, s);
+        }
+      }
+      if (e != cudaSuccess) return cuda_fail(e, "swap copy");
+    }
+  }
+  return PA_OK;
+}
+
+}  // namespace
+
+pa_status pa_swap_bytes(const pa_pool* p, int32_t n_tokens, size_t* bytes) {
+  g_last_error.clear();
+  if (!p || !bytes || n_tokens < 0) return fail(PA_ERR_INVALID_ARG, "null argument or negative length");
+  *bytes = swap_image_bytes(p->d, n_tokens);
+  return PA_OK;
+}
+
+pa_status pa_swap_out(pa_pool* p, int32_t seq, void* host, size_t host_bytes, void* stream) {
+  g_last_error.clear();
+  if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
+  if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
+  pa_status st = seq_arg(p, seq);
+  if (st != PA_OK) return st;
+  if (!p->bm->active(seq)) return fail(PA_ERR_NO_SEQ, "pa_swap_out: no such sequence");
+  DeviceGuard guard(p->d.device);
+  if (!guard.ok) return fail(PA_ERR_CUDA, "cannot select the pool's device");
+  st = check_host_image(host, host_bytes, swap_image_bytes(p->d, p->bm->len(seq)));
+  if (st != PA_OK) return st;
+  const std::vector<int32_t> table = p->bm->table(seq);
+  st = swap_copies(p, table, static_cast<char*>(host), true, static_cast<cudaStream_t>(stream));
+  if (st != PA_OK) return st;
+  return bm_status(p->bm->release(seq), "pa_swap_out");
+}
+
+pa_status pa_swap_in(pa_pool* p, int32_t seq, int32_t n_tokens, const void* host, size_t host_bytes,
+                     void* stream) {
+  g_last_error.clear();
+  if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
+  if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
+  pa_status st = seq_arg(p, seq);
+  if (st != PA_OK) return st;
+  if (n_tokens < 0) return fail(PA_ERR_INVALID_ARG, "negative length");
+  if (p->bm->active(seq)) return fail(PA_ERR_SEQ_EXISTS, "pa_swap_in: sequence exists");
+  DeviceGuard guard(p->d.device);
+  if (!guard.ok) return fail(PA_ERR_CUDA, "cannot select the pool's device");
+  st = check_host_image(host, host_bytes, swap_image_bytes(p->d, n_tokens));
+  if (st != PA_OK) return st;
+  p->cows.clear();
+  st = bm_status(p->bm->reserve(seq, n_tokens, &p->cows), "pa_swap_in");
+  if (st != PA_OK) return st;
+  st = swap_copies(p, p->bm->table(seq), static_cast<char*>(const_cast<void*>(host)), false,
+                   static_cast<cudaStream_t>(stream));
+  if (st != PA_OK) p->bm->release(seq);
+  return st;
+}
+
 pa_status pa_append_kv(pa_pool* p, int32_t layer, int32_t T, const int32_t* seqs,
                        const int32_t* positions, const void* k_new, const void* v_new,
                        void* stream) {
