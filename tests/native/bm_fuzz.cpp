@@ -1,0 +1,119 @@
+// Random-operation fuzz of the host block manager, built with the address and
+// undefined-behaviour sanitizers by tests/test_host_sanitized.py.  After every
+// operation it checks the pool invariants from the block manager's own
+// accessors: each block is free, cached or referenced, and exactly one of
+// these; reference counts equal the table entries that name a block; cached
+// blocks are registered and unreferenced; a match never exceeds the prompt's
+// whole blocks and its blocks equal those the new sequence receives.
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <random>
+#include <vector>
+
+#include "block_manager.h"
+
+namespace {
+
+int fails = 0;
+// Records a failed check; the loops stop at the first one.
+#define CHECK(c)                                                            \
+  do {                                                                      \
+    if (!(c) && fails++ == 0)                                               \
+      std::fprintf(stderr, "check failed at line %d: %s\n", __LINE__, #c); \
+  } while (0)
+
+void check(const pa::BlockManager& bm) {
+  const int nb = bm.num_blocks();
+  std::vector<int> refs(nb, 0), seen(nb, 0);
+  for (int s = 0; s < bm.max_seqs(); ++s) {
+    if (!bm.active(s)) continue;
+    const auto& t = bm.table(s);
+    CHECK(static_cast<int64_t>(t.size()) ==
+          (static_cast<int64_t>(bm.len(s)) + bm.block_size() - 1) / bm.block_size());
+    for (int b : t) {
+      CHECK(b >= 0 && b < nb);
+      ++refs[b];
+    }
+  }
+  std::vector<int32_t> fl, cl;
+  bm.free_list(&fl);
+  bm.cached_list(&cl);
+  CHECK(static_cast<int>(cl.size()) == bm.cached_count());
+  for (int b : fl) {
+    CHECK(b >= 0 && b < nb && !bm.registered(b));
+    ++seen[b];
+  }
+  for (int b : cl) {
+    CHECK(b >= 0 && b < nb && bm.registered(b));
+    ++seen[b];
+  }
+  for (int b = 0; b < nb; ++b) {
+    CHECK(refs[b] == bm.refcount(b));
+    CHECK(seen[b] == (refs[b] == 0 ? 1 : 0));
+  }
+}
+
+}  // namespace
+
+int main(int argc, char** argv) {
+  const int seeds = argc > 1 ? std::atoi(argv[1]) : 20;
+  for (int seed = 0; seed < seeds && fails == 0; ++seed) {
+    std::mt19937 g(seed);
+    const int B = (seed % 2) ? 32 : 16, nb = 24 + seed * 7, max_seqs = 12, mbps = 24;
+    std::vector<int32_t> order(nb);
+    for (int i = 0; i < nb; ++i) order[i] = i;
+    std::shuffle(order.begin(), order.end(), g);
+    pa::BlockManager bm(nb, B, max_seqs, mbps, order.data());
+    const int vocab = 1 + seed % 4;
+    std::vector<std::vector<int32_t>> hist(max_seqs), done;
+    std::vector<pa::CowPair> cows;
+    for (int it = 0; it < 3000 && fails == 0; ++it) {
+      const int s = static_cast<int>(g() % max_seqs);
+      const int op = static_cast<int>(g() % 100);
+      if (op < 25 && !bm.active(s)) {  // new prompt, maybe a continuation
+        std::vector<int32_t> toks = (!done.empty() && g() % 2) ? done[g() % done.size()]
+                                                               : std::vector<int32_t>();
+        const int extra = static_cast<int>(g() % (3 * B));
+        for (int k = 0; k < extra; ++k) toks.push_back(static_cast<int32_t>(g() % vocab));
+        if (static_cast<int>(toks.size()) > mbps * B) toks.resize(mbps * B);
+        std::vector<int32_t> hit;
+        const int m = bm.match_prefix(static_cast<int32_t>(toks.size()), toks.data(), &hit);
+        CHECK(m * B <= static_cast<int>(toks.size()));
+        int32_t cached = -1;
+        if (bm.reserve_prefix(s, static_cast<int32_t>(toks.size()), toks.data(), &cached) == pa::kOk) {
+          CHECK(cached == m * B);
+          for (int j = 0; j < m; ++j) CHECK(bm.table(s)[j] == hit[j]);
+          hist[s] = toks;
+          CHECK(bm.register_prefix(s, static_cast<int32_t>(toks.size()), toks.data()) == pa::kOk);
+        }
+      } else if (op < 35 && bm.active(s)) {  // fork
+        const int c = static_cast<int>(g() % max_seqs);
+        if (!bm.active(c) && bm.fork(s, c) == pa::kOk) hist[c] = hist[s];
+      } else if (op < 75 && bm.active(s)) {  // grow
+        const int grow = 1 + static_cast<int>(g() % (2 * B));
+        const int n = bm.len(s) + grow;
+        cows.clear();
+        if (n <= mbps * B && bm.reserve(s, n, &cows) == pa::kOk) {
+          for (int k = 0; k < grow; ++k) hist[s].push_back(static_cast<int32_t>(g() % vocab));
+          if (g() % 3 == 0)
+            CHECK(bm.register_prefix(s, static_cast<int32_t>(hist[s].size()), hist[s].data()) == pa::kOk);
+        }
+      } else if (op < 90 && bm.active(s)) {  // finish
+        CHECK(bm.release(s) == pa::kOk);
+        done.push_back(hist[s]);
+        if (done.size() > 16) done.erase(done.begin());
+      } else if (bm.active(s) && bm.len(s) > 0) {  // a write must avoid shared and cached blocks
+        int64_t slot = 0;
+        const int pos = static_cast<int>(g() % bm.len(s));
+        const int b = bm.table(s)[pos / B];
+        const pa::Status st = bm.slot(s, pos, &slot);
+        CHECK((st == pa::kSharedBlock) == (bm.refcount(b) > 1 || bm.registered(b)));
+      }
+      check(bm);
+    }
+  }
+  if (fails) return 1;
+  std::printf("ok\n");
+  return 0;
+}
