@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-swap", action="store_true",
+                    help="skip the swap-out / swap-in transfer measurement")
     ap.add_argument("--separate-append", action="store_true",
                     help="append with pa_append_kv and decode with pa_decode_attention (two launches "
                          "per layer) instead of the fused pa_decode_attention_append")
@@ -493,7 +495,57 @@ def run_ours(a, rank, world, local_rank):
         line["graph_batch"] = graph_batch(r, 1000)
     if rank == 0 and not a.no_cpu:
         line["cpu_baseline"] = cpu_baseline(w, a.cpu_seconds, lens0)
+    if rank == 0 and not a.no_swap:
+        line["swap"] = swap_probe(device)
     return line
+
+
+def swap_probe(device, reps=5):
+    """Host transfer of one preempted sequence, outside the timed step: the
+    1,525-token request of "Managing the KV Cache", Hands-On Exercise, in a pool
+    of its 80-layer, 8-KV-head bf16 model, swapped out to pinned host memory and
+    back (pa_swap_out / pa_swap_in: whole allocated blocks, every layer, K and
+    V), timed with CUDA events on the launching stream after one warm-up round
+    trip.  Reports the allocated bytes moved, the useful-state bytes they hold
+    and the achieved GB/s each way; an error is reported, not raised."""
+    import torch
+    import pagedattention_decode_03_b200 as pa
+    n, L, H = 1525, 80, 8
+    nb = -(-n // 16)
+    pool = img = None
+    try:
+        pool = pa.pa_pool_create(num_layers=L, num_kv_heads=H, block_size=16, num_blocks=nb,
+                                 max_seqs=1, max_blocks_per_seq=nb, kv_dtype="bf16", device=device)
+        pa.pa_alloc_blocks(pool, 0, n)
+        size = pa.pa_swap_bytes(pool, n)
+        img = torch.empty(size, dtype=torch.uint8, pin_memory=True)
+        s = torch.cuda.current_stream(device)
+        t_out, t_in = [], []
+        for rep in range(reps + 1):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            ev[0].record(s)
+            pa.pa_swap_out(pool, 0, img, s)
+            ev[1].record(s)
+            pa.pa_swap_in(pool, 0, n, img, s)
+            ev[2].record(s)
+            torch.cuda.synchronize(device)
+            if rep:
+                t_out.append(ev[0].elapsed_time(ev[1]))
+                t_in.append(ev[1].elapsed_time(ev[2]))
+        out_ms, in_ms = statistics.median(t_out), statistics.median(t_in)
+        return {"tokens": n, "layers": L, "kv_heads": H, "dtype": "bf16",
+                "allocated_bytes": size, "useful_bytes": n * 2 * L * H * 128 * 2,
+                "out_ms": round(out_ms, 3), "in_ms": round(in_ms, 3),
+                "out_gbs": round(size / (out_ms * 1e-3) / 1e9, 2),
+                "in_gbs": round(size / (in_ms * 1e-3) / 1e9, 2),
+                "host_memory": "pinned", "reps": reps}
+    except Exception as ex:  # a failed probe must not cost the benchmark line
+        return {"error": f"{type(ex).__name__}: {ex}"[:300]}
+    finally:
+        if pool is not None:
+            torch.cuda.synchronize(device)
+            pa.pa_pool_destroy(pool)
+        del img
 
 
 def graph_batch(r, reps):
