@@ -313,6 +313,27 @@ def test_errors_leave_state_unchanged():
     assert before == (pa.pa_get_free_list(p.pool), pa.pa_get_refcounts(p.pool))
 
 
+def test_empty_calls_launch_nothing_and_change_nothing():
+    """Zero sequences or tokens: every call succeeds, launches no kernel and
+    leaves tables, counts, free list and cache as they were."""
+    w = workload("tiny")
+    p = Pair(w)
+    p.prefill()
+    before = (pa.pa_get_free_list(p.pool), pa.pa_get_refcounts(p.pool), pa.pa_launch_count(p.pool))
+    q = torch.zeros((0, 8, 128), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((0, 2, 128), dtype=torch.bfloat16, device="cuda")
+    for part in (0, -1, 512):
+        pa.pa_decode_attention(p.pool, 0, [], q, torch.empty_like(q), w.scale, part)
+        pa.pa_decode_attention_append(p.pool, 0, [], kv, kv, q, torch.empty_like(q), w.scale, part)
+    pa.pa_append_kv(p.pool, 0, [], [], kv, kv)
+    assert pa.pa_alloc_blocks_n(p.pool, [], []) == 0
+    torch.cuda.synchronize()
+    assert before == (pa.pa_get_free_list(p.pool), pa.pa_get_refcounts(p.pool), pa.pa_launch_count(p.pool))
+    p.check_metadata()
+    p.check_cache(0)
+    assert p.device_errors() == 0
+
+
 @pytest.mark.parametrize("partition", [512, 0, -1])
 def test_fp8_long_context_reduced(partition):
     """FP8-E4M3 KV with per-(layer, head) scales, 64 q / 8 KV heads, 8 sequences
