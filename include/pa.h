@@ -86,7 +86,8 @@ typedef struct {
   int32_t num_layers;
   int32_t num_kv_heads;
   int32_t head_dim;           /* must be 128 */
-  int32_t block_size;         /* tokens per block: 16 (32 accepted by the block manager only) */
+  int32_t block_size;         /* tokens per block: 16 or 32; decode takes 16 only (32 serves
+                                 reservation, append, copy-on-write, swapping, prefix cache) */
   int32_t num_blocks;         /* physical blocks in the pool */
   int32_t max_seqs;           /* sequence ids are 0 .. max_seqs-1 */
   int32_t max_blocks_per_seq; /* block-table capacity of one sequence */
