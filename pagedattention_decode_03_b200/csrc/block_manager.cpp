@@ -257,23 +257,36 @@ Status BlockManager::register_prefix(int32_t seq, int32_t n, const int32_t* toke
   if (!s.active) return kNoSeq;
   if (n > s.len) return kInvalidArg;
   const int32_t m = n / block_size_;
-  // validate: a block registered already must hold this very prefix
-  int32_t node = -1;
-  bool path = true;
+  const size_t row = sizeof(int32_t) * block_size_;
+  // Validate: a block registered already must hold this very prefix.  Its node
+  // is known, so that is a parent and token comparison (nodes are unique per
+  // (parent, tokens)); only unregistered blocks need the index.
+  int32_t node = -1;  // node of the prefix before block i (-1: the empty prefix)
+  bool path = true;   // that node exists
   for (int32_t i = 0; i < m; ++i) {
     const int32_t* toks = tokens + static_cast<int64_t>(i) * block_size_;
-    node = path ? find_child(node, toks) : -1;
-    path = node >= 0;
     const int32_t bn = block_node_[s.table[i]];
-    if (bn >= 0 && bn != node) return kInvalidArg;
+    if (bn >= 0) {
+      if (!path || nodes_[bn].parent != node ||
+          std::memcmp(&node_tokens_[static_cast<size_t>(bn) * block_size_], toks, row) != 0)
+        return kInvalidArg;
+      node = bn;
+    } else {
+      node = path ? find_child(node, toks) : -1;
+      path = node >= 0;
+    }
   }
   node = -1;
   for (int32_t i = 0; i < m; ++i) {
+    const int32_t b = s.table[i];
+    if (block_node_[b] >= 0) {  // validated above: the node of this prefix
+      node = block_node_[b];
+      continue;
+    }
     const int32_t* toks = tokens + static_cast<int64_t>(i) * block_size_;
     int32_t c = find_child(node, toks);
     if (c < 0) c = add_child(node, toks);
-    const int32_t b = s.table[i];
-    if (nodes_[c].block < 0 && block_node_[b] < 0) {
+    if (nodes_[c].block < 0) {
       nodes_[c].block = b;
       block_node_[b] = c;
     }
