@@ -360,8 +360,12 @@ class PagedKVOracle:
             return (Status.NO_SEQ if 0 <= seq < self.max_seqs else Status.INVALID_ARG), None, 0
         table, n = self.tables[seq], self.lens[seq]
         layers = sorted(self.k)
-        image = np.stack([np.stack([np.stack([cache[layer][b] for layer in layers]) for b in table])
-                          for cache in (self.k, self.v)])
+        store = np.uint8 if self.kv_dtype == "fp8_e4m3" else np.uint16
+        image = np.zeros((2, len(table), len(layers), self.H, self.B, self.d), store)
+        for c, cache in enumerate((self.k, self.v)):
+            for j, b in enumerate(table):
+                for i, layer in enumerate(layers):
+                    image[c, j, i] = cache[layer][b]
         self.release(seq)
         return Status.OK, image, n
 

@@ -87,8 +87,7 @@ MUTANTS = [
     # swap-out / swap-in
     (paged.PagedKVOracle, "swap_bytes", "(2 * _ceil_div(n_tokens, self.B)", "(_ceil_div(n_tokens, self.B)",
      lambda: swp.test_swap_bytes_are_the_exercise_allocated_bytes()),
-    (paged.PagedKVOracle, "swap_out", "np.stack([np.stack([cache[layer][b] for layer in layers]) for b in table])",
-     "np.stack([np.stack([cache[layer][b] for b in table]) for layer in layers])",
+    (paged.PagedKVOracle, "swap_out", "image[c, j, i] = cache[layer][b]", "image[c, i % len(table), j % len(layers)] = cache[layer][b]",
      lambda: swp.test_image_layout_holds_each_appended_row_at_its_place()),
     (paged.PagedKVOracle, "swap_out", "self.release(seq)", "None",
      lambda: swp.test_round_trip_restores_attention_exactly_and_frees_blocks()),

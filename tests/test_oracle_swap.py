@@ -140,6 +140,15 @@ def test_forked_and_registered_blocks():
     p.o.check_invariants()
 
 
+def test_empty_sequence_swaps_an_empty_image():
+    p = Pool(seed=4)
+    assert p.o.reserve(0, 0) == Status.OK
+    st, img, n = p.o.swap_out(0)
+    assert st == Status.OK and n == 0 and img.nbytes == p.o.swap_bytes(0, 2) == 0
+    assert p.o.swap_in(0, 0, img) == Status.OK and p.o.lens[0] == 0 and p.o.table(0) == []
+    p.o.check_invariants()
+
+
 def test_swap_in_without_room_changes_nothing():
     p = Pool(nb=8, seed=3)
     p.grow(0, 64)                                   # 4 blocks
