@@ -138,4 +138,14 @@ def test_refusals_change_nothing():
     assert e.value.status == pa.PA_ERR_SEQ_EXISTS
     P.check_metadata()
     P.check_cache(0)
+    # an empty sequence swaps an empty image, with no copy
+    pa.pa_alloc_blocks(P.pool, 5, 0)
+    assert P.oracle.reserve(5, 0) == Status.OK
+    empty = torch.empty(0, dtype=torch.uint8, pin_memory=True)
+    pa.pa_swap_out(P.pool, 5, empty)
+    st, image, n = P.oracle.swap_out(5)
+    assert st == Status.OK and n == 0 and image.nbytes == 0
+    pa.pa_swap_in(P.pool, 5, 0, empty)
+    assert P.oracle.swap_in(5, 0, image) == Status.OK
+    P.check_metadata()
     assert pa.pa_launch_count(P.pool) > 0 and P.device_errors() == 0
