@@ -31,6 +31,43 @@ void MirrorDeltas::consume(size_t n) {
   for (size_t k = 0; k < idx_.size(); ++k) where_[idx_[k]] = static_cast<int32_t>(k);
 }
 
+void NodeIndex::grow() {
+  std::vector<Slot> old;
+  old.swap(slots_);
+  slots_.assign(old.empty() ? 64 : 2 * old.size(), Slot{0, -1});
+  mask_ = slots_.size() - 1;
+  size_ = 0;
+  for (const Slot& s : old)
+    if (s.node >= 0) insert(s.key, s.node);
+}
+
+void NodeIndex::insert(uint64_t key, int32_t node) {
+  if (2 * (size_ + 1) > slots_.size()) grow();
+  size_t i = key & mask_;
+  while (slots_[i].node >= 0) i = (i + 1) & mask_;
+  slots_[i] = Slot{key, node};
+  ++size_;
+}
+
+void NodeIndex::erase(uint64_t key, int32_t node) {
+  if (slots_.empty()) return;
+  size_t i = key & mask_;
+  while (slots_[i].node >= 0 && !(slots_[i].key == key && slots_[i].node == node)) i = (i + 1) & mask_;
+  if (slots_[i].node < 0) return;
+  // Backward shift: move later entries of the run into the hole whenever
+  // their home slot does not lie cyclically in (hole, entry].
+  for (size_t j = (i + 1) & mask_; slots_[j].node >= 0; j = (j + 1) & mask_) {
+    const size_t home = slots_[j].key & mask_;
+    const bool stays = (i <= j) ? (i < home && home <= j) : (i < home || home <= j);
+    if (!stays) {
+      slots_[i] = slots_[j];
+      i = j;
+    }
+  }
+  slots_[i].node = -1;
+  --size_;
+}
+
 BlockManager::BlockManager(int32_t num_blocks, int32_t block_size, int32_t max_seqs,
                            int32_t max_blocks_per_seq, const int32_t* free_order)
     : num_blocks_(num_blocks), block_size_(block_size), max_seqs_(max_seqs),
@@ -80,17 +117,11 @@ void BlockManager::lru_remove(int32_t b) {
 }
 
 uint64_t BlockManager::node_key(int32_t parent, const int32_t* toks) const {
-  // FNV-1a over the parent id and the tokens, then the MurmurHash3 64-bit
-  // finaliser to spread the bits over the buckets.
+  // FNV-1a over 32-bit words (the parent id, then the tokens), then the
+  // MurmurHash3 64-bit finaliser to spread the bits over the buckets.
   uint64_t h = 0xcbf29ce484222325ull;
-  auto mix = [&h](uint32_t w) {
-    for (int k = 0; k < 4; ++k) {
-      h ^= (w >> (8 * k)) & 0xffu;
-      h *= 0x100000001b3ull;
-    }
-  };
-  mix(static_cast<uint32_t>(parent));
-  for (int32_t i = 0; i < block_size_; ++i) mix(static_cast<uint32_t>(toks[i]));
+  h = (h ^ static_cast<uint32_t>(parent)) * 0x100000001b3ull;
+  for (int32_t i = 0; i < block_size_; ++i) h = (h ^ static_cast<uint32_t>(toks[i])) * 0x100000001b3ull;
   h ^= h >> 33;
   h *= 0xff51afd7ed558ccdull;
   h ^= h >> 33;
@@ -100,15 +131,11 @@ uint64_t BlockManager::node_key(int32_t parent, const int32_t* toks) const {
 }
 
 int32_t BlockManager::find_child(int32_t parent, const int32_t* toks) const {
-  const auto range = index_.equal_range(node_key(parent, toks));
-  for (auto it = range.first; it != range.second; ++it) {
-    const int32_t c = it->second;
-    if (nodes_[c].parent == parent &&
-        std::memcmp(&node_tokens_[static_cast<size_t>(c) * block_size_], toks,
-                    sizeof(int32_t) * block_size_) == 0)
-      return c;
-  }
-  return -1;
+  return index_.find(node_key(parent, toks), [&](int32_t c) {
+    return nodes_[c].parent == parent &&
+           std::memcmp(&node_tokens_[static_cast<size_t>(c) * block_size_], toks,
+                       sizeof(int32_t) * block_size_) == 0;
+  });
 }
 
 int32_t BlockManager::add_child(int32_t parent, const int32_t* toks) {
@@ -125,7 +152,7 @@ int32_t BlockManager::add_child(int32_t parent, const int32_t* toks) {
   nodes_[c] = {parent, -1, 0, key};
   std::memcpy(&node_tokens_[static_cast<size_t>(c) * block_size_], toks,
               sizeof(int32_t) * block_size_);
-  index_.emplace(key, c);
+  index_.insert(key, c);
   if (parent >= 0) ++nodes_[parent].children;
   return c;
 }
@@ -135,13 +162,7 @@ int32_t BlockManager::add_child(int32_t parent, const int32_t* toks) {
 // id never matches a stale key.
 void BlockManager::prune(int32_t node) {
   while (node >= 0 && nodes_[node].block < 0 && nodes_[node].children == 0) {
-    const auto range = index_.equal_range(nodes_[node].key);
-    for (auto it = range.first; it != range.second; ++it) {
-      if (it->second == node) {
-        index_.erase(it);
-        break;
-      }
-    }
+    index_.erase(nodes_[node].key, node);
     const int32_t parent = nodes_[node].parent;
     spare_nodes_.push_back(node);
     if (parent >= 0) --nodes_[parent].children;

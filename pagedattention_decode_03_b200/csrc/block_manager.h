@@ -36,7 +36,6 @@
 #pragma once
 
 #include <cstdint>
-#include <unordered_map>
 #include <vector>
 
 namespace pa {
@@ -72,6 +71,34 @@ class MirrorDeltas {
 
 struct CowPair {
   int32_t src, dst;
+};
+
+// Open-addressing hash table from a 64-bit key to the nodes stored under it
+// (linear probing, load <= 1/2, backward-shift deletion), so inserting and
+// removing a node allocates nothing once the table has grown.
+class NodeIndex {
+ public:
+  void insert(uint64_t key, int32_t node);
+  void erase(uint64_t key, int32_t node);
+  // First node stored under `key` for which `same(node)` holds, or -1.
+  template <class F>
+  int32_t find(uint64_t key, F&& same) const {
+    if (slots_.empty()) return -1;
+    for (size_t i = key & mask_;; i = (i + 1) & mask_) {
+      const Slot& s = slots_[i];
+      if (s.node < 0) return -1;
+      if (s.key == key && same(s.node)) return s.node;
+    }
+  }
+
+ private:
+  struct Slot {
+    uint64_t key;
+    int32_t node;  // -1: empty
+  };
+  void grow();
+  std::vector<Slot> slots_;
+  size_t mask_ = 0, size_ = 0;
 };
 
 class BlockManager {
@@ -155,7 +182,7 @@ class BlockManager {
 
   std::vector<Node> nodes_;
   std::vector<int32_t> node_tokens_, spare_nodes_;
-  std::unordered_multimap<uint64_t, int32_t> index_;  // key -> node
+  NodeIndex index_;                                   // key -> node
   std::vector<int32_t> block_node_;                   // block -> node, or -1
   std::vector<int32_t> lru_prev_, lru_next_;          // -2: not on the list
   int32_t lru_head_ = -1, lru_tail_ = -1, lru_count_ = 0;

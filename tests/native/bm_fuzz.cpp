@@ -4,10 +4,13 @@
 // accessors: each block is free, cached or referenced, and exactly one of
 // these; reference counts equal the table entries that name a block; cached
 // blocks are registered and unreferenced; a match never exceeds the prompt's
-// whole blocks and its blocks equal those the new sequence receives.
+// whole blocks and its blocks equal those the new sequence receives.  Before
+// that, the prefix index's open-addressing table runs against a std::multimap
+// with keys crowded onto three home slots.
 #include <algorithm>
 #include <cstdio>
 #include <cstdlib>
+#include <map>
 #include <random>
 #include <vector>
 
@@ -54,10 +57,42 @@ void check(const pa::BlockManager& bm) {
   }
 }
 
+// The prefix index against a std::multimap, with keys forced onto few home
+// slots (shared low bits) so that probe runs are long, wrap around the table
+// end and are cut by backward-shift deletions.
+void fuzz_node_index(int seed) {
+  std::mt19937_64 g(seed);
+  pa::NodeIndex ix;
+  std::multimap<uint64_t, int32_t> ref;
+  int32_t next = 0;
+  for (int it = 0; it < 4000 && fails == 0; ++it) {
+    const uint64_t key = ((g() % 40) << 20) | (g() % 3) * 61 | 0x3f;  // low bits: 3 homes
+    if (g() % 3 != 0 || ref.empty()) {
+      ix.insert(key, next);
+      ref.emplace(key, next);
+      ++next;
+    } else {
+      auto it_ref = ref.begin();
+      std::advance(it_ref, static_cast<long>(g() % ref.size()));
+      ix.erase(it_ref->first, it_ref->second);
+      ref.erase(it_ref);
+    }
+    // every stored (key, node) is found; a node not stored is not
+    const uint64_t probe = ((g() % 40) << 20) | (g() % 3) * 61 | 0x3f;
+    auto range = ref.equal_range(probe);
+    for (auto r = range.first; r != range.second; ++r) {
+      const int32_t want = r->second;
+      CHECK(ix.find(probe, [&](int32_t n) { return n == want; }) == want);
+    }
+    CHECK(ix.find(probe, [&](int32_t n) { return n == next; }) == -1);
+  }
+}
+
 }  // namespace
 
 int main(int argc, char** argv) {
   const int seeds = argc > 1 ? std::atoi(argv[1]) : 20;
+  for (int seed = 0; seed < 4 && fails == 0; ++seed) fuzz_node_index(seed);
   for (int seed = 0; seed < seeds && fails == 0; ++seed) {
     std::mt19937 g(seed);
     const int B = (seed % 2) ? 32 : 16, nb = 24 + seed * 7, max_seqs = 12, mbps = 24;

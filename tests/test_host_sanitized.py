@@ -1,7 +1,8 @@
 """The host block manager (free list, reference counts, copy-on-write,
-prefix trie and cached list) under AddressSanitizer and UBSan: a random-
-operation driver (tests/native/bm_fuzz.cpp) built with g++ against the
-library's own block_manager.cpp checks the pool invariants after every
+prefix trie with its open-addressing index, cached list) under
+AddressSanitizer and UBSan: a random-operation driver (tests/native/bm_fuzz.cpp)
+built with g++ against the library's own block_manager.cpp checks the index
+against std::multimap under crowded keys, then the pool invariants after every
 operation.  No GPU."""
 import os
 import shutil
