@@ -84,6 +84,13 @@ MUTANTS = [
     (paged.PagedKVOracle, "reserve_prefix", "if need > len(self.free) + len(self.cached) - idle:",
      "if need > len(self.free) + len(self.cached):",
      lambda: pfx.test_reusing_every_idle_block_and_needing_one_more_fails_cleanly()),
+    (paged.PagedKVOracle, "register", "if b in self.key_of and self.key_of[b] != self._prefix(tokens, i):",
+     "if False:",
+     lambda: pfx.test_registered_blocks_are_immutable_and_first_registration_wins()),
+    (paged.PagedKVOracle, "reserve_prefix", "self.ref[b] += 1", "pass",
+     lambda: pfx.test_conversations_under_pool_pressure_keep_exact_contents(0)),
+    (paged.PagedKVOracle, "match", "while (m + 1) * self.B <= len(tokens)", "while (m + 2) * self.B <= len(tokens)",
+     lambda: pfx.test_worked_103_token_prompt_reuses_96()),
     # swap-out / swap-in
     (paged.PagedKVOracle, "swap_bytes", "(2 * _ceil_div(n_tokens, self.B)", "(_ceil_div(n_tokens, self.B)",
      lambda: swp.test_swap_bytes_are_the_exercise_allocated_bytes()),
