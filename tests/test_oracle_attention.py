@@ -25,6 +25,17 @@ def _bf16_scalar(bits):
     return struct.unpack("<f", struct.pack("<I", int(bits) << 16))[0]
 
 
+def _fp16_scalar(bits):
+    import struct
+    return struct.unpack("<e", struct.pack("<H", int(bits)))[0]
+
+
+def _scalar(bits, dtype):
+    """One 16-bit pattern to a Python float, by the struct codecs (binary32
+    upper half for bf16, binary16 for fp16), independent of the oracle."""
+    return _bf16_scalar(bits) if dtype == "bf16" else _fp16_scalar(bits)
+
+
 def build(lens, H=2, G=2, d=8, B=4, nb=40, kv="bf16", act="bf16", seed=0, order=None):
     g = np.random.default_rng(seed)
     o = PagedKVOracle(num_layers=2, num_kv_heads=H, head_dim=d, block_size=B, num_blocks=nb,
@@ -46,7 +57,7 @@ def build(lens, H=2, G=2, d=8, B=4, nb=40, kv="bf16", act="bf16", seed=0, order=
     return o, q, (k_scale, v_scale)
 
 
-def brute_force(o, layer, lens, q_bits, scale, scales=(None, None)):
+def brute_force(o, layer, lens, q_bits, scale, scales=(None, None), act="bf16"):
     """Scalar-loop attention straight off the pool, one slot at a time."""
     k_scale, v_scale = scales
     n_seq, hq, d = q_bits.shape
@@ -56,7 +67,7 @@ def brute_force(o, layer, lens, q_bits, scale, scales=(None, None)):
     for s in range(n_seq):
         for qh in range(hq):
             h = qh // G
-            qv = [_bf16_scalar(q_bits[s, qh, j]) for j in range(d)]
+            qv = [_scalar(q_bits[s, qh, j], act) for j in range(d)]
             logits = []
             for t in range(lens[s]):
                 blk = o.tables[s][t // o.B]
@@ -64,7 +75,7 @@ def brute_force(o, layer, lens, q_bits, scale, scales=(None, None)):
                 if o.kv_dtype == "fp8_e4m3":
                     kv = [float(fp8.decode([row[j]])[0]) * float(k_scale[layer][h]) for j in range(d)]
                 else:
-                    kv = [_bf16_scalar(row[j]) for j in range(d)]
+                    kv = [_scalar(row[j], o.kv_dtype) for j in range(d)]
                 acc = 0.0
                 for j in range(d):
                     acc += qv[j] * kv[j]
@@ -79,7 +90,7 @@ def brute_force(o, layer, lens, q_bits, scale, scales=(None, None)):
                     if o.kv_dtype == "fp8_e4m3":
                         vj = float(fp8.decode([row[j]])[0]) * float(v_scale[layer][h])
                     else:
-                        vj = _bf16_scalar(row[j])
+                        vj = _scalar(row[j], o.kv_dtype)
                     out[s, qh, j] += w[t] / tot * vj
     return out
 
@@ -91,6 +102,16 @@ def test_matches_scalar_brute_force(G):
     for layer in (0, 1):
         got = o.attention(layer, range(len(lens)), q, "bf16", 0.35)
         want = brute_force(o, layer, lens, q, 0.35)
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("G", [1, 4])
+def test_fp16_matches_scalar_brute_force(G):
+    lens = [1, 6, 11]
+    o, q, _ = build(lens, G=G, kv="fp16", act="fp16", seed=20 + G)
+    for layer in (0, 1):
+        got = o.attention(layer, range(len(lens)), q, "fp16", 0.35)
+        want = brute_force(o, layer, lens, q, 0.35, act="fp16")
         np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
 
 

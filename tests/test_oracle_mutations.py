@@ -12,10 +12,11 @@ import numpy as np
 import pytest
 
 import oracle
-from oracle import fp8, paged, sizing
+from oracle import fp8, numerics, paged, sizing
 
 import test_oracle_attention as att
 import test_oracle_fp8 as tf8
+import test_oracle_numerics as tnum
 import test_oracle_pool as pool
 import test_oracle_prefix as pfx
 import test_oracle_swap as swp
@@ -65,6 +66,17 @@ MUTANTS = [
      lambda: pool.test_invalid_calls()),
     (paged.PagedKVOracle, "append", "self.k[layer][b, :, o, :] = k_bits[t]", "self.k[layer][b, :, o - 1, :] = k_bits[t]",
      lambda: pool.test_append_writes_the_slot_and_nothing_else()),
+    # fp16 storage widened as if it were bf16 (caught by the definition and by
+    # the fp16 brute force, which decodes with the struct binary16 codec)
+    (numerics, "bits_to_f64", "return b.view(np.float16).astype(np.float64)",
+     "return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)",
+     lambda: tnum.test_fp16_values_from_definition()),
+    (numerics, "bits_to_f64", "return b.view(np.float16).astype(np.float64)",
+     "return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)",
+     lambda: att.test_fp16_matches_scalar_brute_force(4)),
+    (numerics, "bits_to_f64", "return b.view(np.float16).astype(np.float64)",
+     "return b.view(np.float16).astype(np.float32).astype(np.float64) * (1 + 2.0 ** -11)",
+     lambda: tnum.test_named_fp16_values()),
     # block-granular prefix cache
     (paged.PagedKVOracle, "_prefix", "tokens[: (i + 1) * self.B]", "tokens[i * self.B : (i + 1) * self.B]",
      lambda: pfx.test_conversations_under_pool_pressure_keep_exact_contents(0)),
@@ -120,7 +132,11 @@ def test_planted_mistake_is_caught(case, monkeypatch, golden_dir):
     target, name, old, new, pin = MUTANTS[case]
     real = getattr(target, name)
     func = real if inspect.isfunction(real) else real.__func__
-    monkeypatch.setattr(target, name, _mutated(func, old, new))
+    mutant = _mutated(func, old, new)
+    monkeypatch.setattr(target, name, mutant)
+    if target is numerics:
+        # the pool model holds its own reference to the widening function
+        monkeypatch.setattr(paged, name, mutant)
     if target is sizing:
         # sizing helpers call each other through module globals, so the
         # capacity pins see the mutant too
