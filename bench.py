@@ -4,9 +4,11 @@ One step = one decode step of the workload: reserve one more slot per
 sequence (block manager; a block on boundary crossings, copy-on-write where
 a shared tail is written), then for every layer append the step's K/V row
 per sequence and run decode attention for every sequence -- all through the
-C ABI (libpa.so).  Default workload: the 8B-class GQA layer (64 sequences,
-lengths uniform in [128, 4096], 32 query / 8 KV heads, head_dim 128, bf16,
-16-token blocks, shuffled pool sized 1.25x the need at the end of the run).
+C ABI (libpa.so).  Default workload: the 70B-class GQA model of "Managing
+the KV Cache" (Worked Capacity Under a 12 GiB KV Budget): 80 layers, 64 query /
+8 KV heads, head_dim 128, bf16, 16-token blocks, 47 sequences of 825 tokens in
+the 2,457-block pool plus the headroom that lets all of them grow into block
+53, 16 decode steps; `--workload` selects the other configurations.
 
 Metric: achieved HBM GB/s of the step's algorithmic bytes (KV read by the
 decode + Q + O + block-table entries + appended rows read and written),
@@ -47,9 +49,10 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: the workload's own decode step count)")
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="gqa8b",
+    ap.add_argument("--workload", default="gqa70b_headroom",
                     choices=["tiny", "gqa8b", "gqa70b_headroom", "mha7b_share", "fp8_long"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--partition", type=int, default=None,
@@ -63,6 +66,8 @@ def parse():
     ap.add_argument("--separate-append", action="store_true",
                     help="append with pa_append_kv and decode with pa_decode_attention (two launches "
                          "per layer) instead of the fused pa_decode_attention_append")
+    ap.add_argument("--decode-path", default="auto", choices=["auto", "warp", "tcgen05"],
+                    help="decode kernel for a query group of 8 over 16-bit KV (pa_set_decode_path)")
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling: keep only the first N layers (a smaller case of the same "
                          "kernels; the JSON line then names the reduced workload)")
@@ -70,6 +75,9 @@ def parse():
 
 
 DEFAULT_STEPS = {"tiny": 1, "gqa8b": 100, "gqa70b_headroom": 16, "mha7b_share": 64, "fp8_long": 1}
+# timed steps when --steps is not given: the workload's decode steps, and
+# enough launches for a stable mean where a workload has a single step
+BENCH_STEPS = {"tiny": 100, "gqa8b": 100, "gqa70b_headroom": 16, "mha7b_share": 64, "fp8_long": 20}
 
 
 def pool_steps(a):
@@ -245,9 +253,11 @@ class Runner:
         L, H, Hq, d = w.num_layers, w.num_kv_heads, w.num_q_heads, w.head_dim
         kw = {}
         if w.kv_dtype == "fp8_e4m3":
-            # calibration: amax/448 of N(0,1) data per (layer, head), computed on the
-            # prefill the replica writes (see prefill below)
-            self.amax = torch.zeros((L, H), dtype=torch.float32, device=device)
+            # calibration as the tests use it: separate K and V scales per
+            # (layer, head), amax/448 over every value the replica writes
+            # (prefill and the step inputs below)
+            amax_k = torch.zeros((L, H), dtype=torch.float32, device=device)
+            amax_v = torch.zeros((L, H), dtype=torch.float32, device=device)
         self.scales = None
         # prefill data per (layer, seq) generated on the device
         self.prefill_data = {}
@@ -257,12 +267,21 @@ class Runner:
                 v = torch.randn((n, H, d), generator=gen, device=device, dtype=torch.float32).to(act)
                 self.prefill_data[(layer, s)] = (k, v)
                 if w.kv_dtype == "fp8_e4m3":
-                    self.amax[layer] = torch.maximum(self.amax[layer], torch.maximum(
-                        k.float().abs().amax(dim=(0, 2)), v.float().abs().amax(dim=(0, 2))))
+                    amax_k[layer] = torch.maximum(amax_k[layer], k.float().abs().amax(dim=(0, 2)))
+                    amax_v[layer] = torch.maximum(amax_v[layer], v.float().abs().amax(dim=(0, 2)))
+        # per-step inputs: a few distinct sets, cycled
+        n = len(w.seq_ids)
+        self.nsets = 4
+        self.q = [torch.randn((L, n, Hq, d), generator=gen, device=device).to(act) for _ in range(self.nsets)]
+        self.kn = [torch.randn((L, n, H, d), generator=gen, device=device).to(act) for _ in range(self.nsets)]
+        self.vn = [torch.randn((L, n, H, d), generator=gen, device=device).to(act) for _ in range(self.nsets)]
         if w.kv_dtype == "fp8_e4m3":
-            ks = (self.amax * 1.02 / 448.0).float().contiguous()
-            inv = (1.0 / ks).float().contiguous()
-            self.scales = (ks, ks.clone(), inv, inv.clone())
+            for kn, vn in zip(self.kn, self.vn):
+                amax_k = torch.maximum(amax_k, kn.float().abs().amax(dim=(1, 3)))
+                amax_v = torch.maximum(amax_v, vn.float().abs().amax(dim=(1, 3)))
+            ks = (amax_k / 448.0).float().contiguous()
+            vs = (amax_v / 448.0).float().contiguous()
+            self.scales = (ks, vs, (1.0 / ks).float().contiguous(), (1.0 / vs).float().contiguous())
             kw = dict(k_scale=self.scales[0], v_scale=self.scales[1],
                       k_inv_scale=self.scales[2], v_inv_scale=self.scales[3])
         order = w.free_order()
@@ -272,21 +291,15 @@ class Runner:
             act_dtype=w.act_dtype, free_order=order, device=device,
             min_partition_tokens=min(512, partition) if partition and partition > 0 else 0, **kw)
         for s in sorted(w.prefill_lens):
-            n = w.prefill_lens[s]
-            pa.pa_alloc_blocks(self.pool, s, n)
+            plen = w.prefill_lens[s]
+            pa.pa_alloc_blocks(self.pool, s, plen)
             for layer in range(L):
                 k, v = self.prefill_data.pop((layer, s))
-                pa.pa_append_kv(self.pool, layer, [s] * n, list(range(n)), k, v)
+                pa.pa_append_kv(self.pool, layer, [s] * plen, list(range(plen)), k, v)
         for parent, child in w.forks:
             pa.pa_fork_cow(self.pool, parent, child)
         torch.cuda.synchronize(device)
-        # per-step inputs: a few distinct sets, cycled
-        n = len(w.seq_ids)
-        self.nsets = 4
-        self.q = [torch.randn((L, n, Hq, d), generator=gen, device=device).to(act) for _ in range(self.nsets)]
-        self.kn = [torch.randn((L, n, H, d), generator=gen, device=device).to(act) for _ in range(self.nsets)]
-        self.vn = [torch.randn((L, n, H, d), generator=gen, device=device).to(act) for _ in range(self.nsets)]
-        self.out = torch.empty((L, n, Hq, d), dtype=act, device=device)
+        self.out = torch.empty((L, len(w.seq_ids), Hq, d), dtype=act, device=device)
         # per-layer device addresses, computed once (no tensor views inside the timed loop)
         self._ptrs = {}
         self.seqs = np.asarray(w.seq_ids, np.int32)
@@ -322,25 +335,24 @@ class Runner:
             raise RuntimeError(f"pa_alloc_blocks_n: {self.pa.pa_last_error()}")
         pos = self.lens.ctypes.data_as(self.i32p)
         scale = ctypes.c_float(w.scale)
+        if dec_events is not None:   # the layer loop, back to back: launch overlap intact
+            dec_events[0].record()
         for layer in range(w.num_layers):
             pq, pk, pv, po = ptrs[layer]
             if not self.fused:
                 st = L.pa_append_kv(self.pool.handle, layer, n, sp, pos, pk, pv, stream)
                 if st != 0:
                     raise RuntimeError(f"pa_append_kv: {self.pa.pa_last_error()}")
-            if dec_events is not None:
-                dec_events[0].record()
             if self.fused:   # append of the step's token and decode in one launch
                 st = L.pa_decode_attention_append(self.pool.handle, layer, n, sp, pk, pv, w.num_q_heads,
                                                   pq, po, scale, self.partition, stream)
             else:
                 st = L.pa_decode_attention(self.pool.handle, layer, n, sp, w.num_q_heads, pq, po, scale,
                                            self.partition, stream)
-            if dec_events is not None:
-                dec_events[1].record()
-                dec_events = None  # time the first layer's decode only
             if st != 0:
                 raise RuntimeError(f"pa_decode_attention: {self.pa.pa_last_error()}")
+        if dec_events is not None:
+            dec_events[1].record()
         self.lens = new
         self.step_idx += 1
 
@@ -354,6 +366,10 @@ def reduce_ranks(vals, op, device, world):
     torch.distributed.all_reduce(
         t, op=torch.distributed.ReduceOp.MAX if op == "max" else torch.distributed.ReduceOp.SUM)
     return [float(x) for x in t.tolist()]
+
+
+def steps_of(a):
+    return BENCH_STEPS[a.workload] if a.steps is None else a.steps
 
 
 def run_ours(a, rank, world, local_rank):
@@ -370,6 +386,7 @@ def run_ours(a, rank, world, local_rank):
     partition = w.partition_tokens if a.partition is None else a.partition
     r = Runner(w, device, partition, a.seed + rank)
     r.fused = not a.separate_append
+    r.pa.pa_set_decode_path(r.pool, a.decode_path)
     stream_obj = torch.cuda.current_stream(device)
     stream = ctypes.c_void_p(stream_obj.cuda_stream)
     pa = r.pa
@@ -381,12 +398,16 @@ def run_ours(a, rank, world, local_rank):
     lens0 = r.lens_dict()
     bytes_step = [step_bytes(w, {s: lens0[s] + i for s in lens0}) for i in range(a.steps)]
     total_bytes = sum(b for b, _ in bytes_step)
-    dec_bytes = [d for _, d in bytes_step]
+    # bytes of the kernels inside the layer loop: the decode plus, when fused,
+    # the step's append (separate appends are launched inside the loop too)
+    loop_bytes = [b for b, _ in bytes_step]
     logical = sum(logical_decode_bytes(w, {s: lens0[s] + i for s in lens0}) for i in range(a.steps))
-    # the decode launch is timed on every 4th step: events between two launches
-    # keep the second from starting early, so the other steps run without them
+    # the layer loop of every step is bracketed by two events: inside it the
+    # decode launches run back to back, each overlapping its neighbour's
+    # prologue as in an untimed step (an event between two launches would
+    # stop the second from starting early)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          if i % 4 == 0 else None for i in range(a.steps)]
+          for _ in range(a.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = pa.pa_launch_count(r.pool)
     if world > 1:
@@ -402,7 +423,7 @@ def run_ours(a, rank, world, local_rank):
         torch.cuda.synchronize(device)
     launches = pa.pa_launch_count(r.pool) - launches0
     ms = start.elapsed_time(end)
-    dec_ms = [e[0].elapsed_time(e[1]) for e in ev if e is not None]
+    loop_ms = [e[0].elapsed_time(e[1]) for e in ev]
     bits = pa.pa_check_device_errors(r.pool)
     # every rank takes the same collectives, errors included
     ms, bits = reduce_ranks([ms, float(bits)], "max", device, world)
@@ -446,9 +467,9 @@ def run_ours(a, rank, world, local_rank):
 
     peak, peak_src = peaks()
     value = total_bytes / (ms * 1e-3) / 1e9          # bytes of all ranks / max time
-    dec_mean = statistics.mean(dec_ms)
-    dec_bytes = [d for i, d in enumerate(dec_bytes) if ev[i] is not None]   # the timed launches
-    achieved = statistics.mean(dec_bytes) / w.num_layers / (dec_mean * 1e-3) / 1e9
+    launch_ms = sum(loop_ms) / (len(loop_ms) * w.num_layers)     # per layer
+    launch_bytes = sum(loop_bytes) / (len(loop_bytes) * w.num_layers)
+    achieved = launch_bytes / (launch_ms * 1e-3) / 1e9
     tr = traffic_record(f"{w.name}:decode")
     line = {
         "metric": METRIC,
@@ -467,8 +488,10 @@ def run_ours(a, rank, world, local_rank):
         "data": "synthetic (seeded N(0,1) K/V/Q, seeded lengths and block placement)",
         "config": {**describe(w, partition), "parallelism": f"replicas x{world} (no exchange step)"},
         "roofline": {
-            "kernel": ("decode attention" + (" with the step's append fused" if r.fused else "") +
-                       " (decode kernel, + reduce kernel for fixed partitions), layer 0 of every 4th step"),
+            "kernel": ("decode attention" + (" with the step's append fused" if r.fused else
+                                             ", after a separate append launch") +
+                       " (decode kernel, + reduce kernel for fixed partitions): every step's layer "
+                       "loop timed as a whole, per layer"),
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peak,
@@ -477,11 +500,11 @@ def run_ours(a, rank, world, local_rank):
             "frac": round(achieved / peak, 4),
             # ncu dram read+write of one captured launch of this kernel, scaled to this
             # launch's algorithmic bytes (same workload, a few tokens shorter)
-            "traffic": (int(tr["ratio_to_algorithmic"] * statistics.mean(dec_bytes) / w.num_layers)
-                        if tr else None),
+            "traffic": (int(tr["ratio_to_algorithmic"] * launch_bytes) if tr else None),
             "traffic_over_algorithmic": tr["ratio_to_algorithmic"] if tr else None,
-            "algorithmic_bytes_per_launch": int(statistics.mean(dec_bytes) / w.num_layers),
-            "launch_ms": round(dec_mean, 5),
+            "algorithmic_bytes_per_launch": int(launch_bytes),
+            "launch_ms": round(launch_ms, 5),
+            "ncu_launch_us": tr.get("duration_us") if tr else None,
         },
         "logical_decode_gbs": round(world * logical / (ms * 1e-3) / 1e9, 1),
         "gpu_launches": int(launches),
@@ -491,6 +514,7 @@ def run_ours(a, rank, world, local_rank):
     }
     line["config"]["append"] = ("fused into the decode launch (pa_decode_attention_append)" if r.fused
                                 else "separate launch (pa_append_kv)")
+    line["config"]["decode_kernel"] = pa.pa_last_decode_kernel(r.pool)
     if w.name == "tiny":
         line["graph_batch"] = graph_batch(r, 1000)
     if rank == 0 and not a.no_cpu:
@@ -533,11 +557,35 @@ def swap_probe(device, reps=5):
                 t_out.append(ev[0].elapsed_time(ev[1]))
                 t_in.append(ev[1].elapsed_time(ev[2]))
         out_ms, in_ms = statistics.median(t_out), statistics.median(t_in)
+        # the roofline of a swap is the host link: one contiguous copy of the
+        # same bytes each way between a device buffer and the pinned image
+        dev = torch.empty(size, dtype=torch.uint8, device=device)
+        l_out, l_in = [], []
+        for rep in range(reps + 1):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            ev[0].record(s)
+            img.copy_(dev, non_blocking=True)
+            ev[1].record(s)
+            dev.copy_(img, non_blocking=True)
+            ev[2].record(s)
+            torch.cuda.synchronize(device)
+            if rep:
+                l_out.append(ev[0].elapsed_time(ev[1]))
+                l_in.append(ev[1].elapsed_time(ev[2]))
+        del dev
+        link_out = size / (statistics.median(l_out) * 1e-3) / 1e9
+        link_in = size / (statistics.median(l_in) * 1e-3) / 1e9
+        out_gbs, in_gbs = size / (out_ms * 1e-3) / 1e9, size / (in_ms * 1e-3) / 1e9
         return {"tokens": n, "layers": L, "kv_heads": H, "dtype": "bf16",
                 "allocated_bytes": size, "useful_bytes": n * 2 * L * H * 128 * 2,
                 "out_ms": round(out_ms, 3), "in_ms": round(in_ms, 3),
-                "out_gbs": round(size / (out_ms * 1e-3) / 1e9, 2),
-                "in_gbs": round(size / (in_ms * 1e-3) / 1e9, 2),
+                "out_gbs": round(out_gbs, 2), "in_gbs": round(in_gbs, 2),
+                "roofline": {"bound": "host link", "unit": "GB/s",
+                             "peak_out": round(link_out, 2), "peak_in": round(link_in, 2),
+                             "peak_source": "measured: one contiguous cudaMemcpyAsync of the same "
+                                            "bytes each way, device buffer <-> pinned host",
+                             "frac_out": round(out_gbs / link_out, 4),
+                             "frac_in": round(in_gbs / link_in, 4)},
                 "host_memory": "pinned", "reps": reps}
     except Exception as ex:  # a failed probe must not cost the benchmark line
         return {"error": f"{type(ex).__name__}: {ex}"[:300]}
@@ -699,6 +747,7 @@ def run_reference(a):
 
 def main():
     a = parse()
+    a.steps = steps_of(a)
     if a.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     rank = int(os.environ.get("RANK", "0"))

@@ -86,8 +86,8 @@ typedef struct {
   int32_t num_layers;
   int32_t num_kv_heads;
   int32_t head_dim;           /* must be 128 */
-  int32_t block_size;         /* tokens per block: 16 or 32; decode takes 16 only (32 serves
-                                 reservation, append, copy-on-write, swapping, prefix cache) */
+  int32_t block_size;         /* tokens per block: 16 or 32 (the decode kernel walks 16-token
+                                 tiles: a 32-token block is read as its two halves) */
   int32_t num_blocks;         /* physical blocks in the pool */
   int32_t max_seqs;           /* sequence ids are 0 .. max_seqs-1 */
   int32_t max_blocks_per_seq; /* block-table capacity of one sequence */
@@ -222,16 +222,34 @@ pa_status pa_decode_attention_append(pa_pool *pool, int32_t layer, int32_t n, co
  * partial results, arrival counters and an error word -- is one
  * static device array of 12 MiB that every GPU loading the library holds
  * until the process exits.  The first call on a device looks up that array's
- * device address (once per device, with the device current); make that first
- * call before any stream capture.  Every call shares the array and clears
- * what must start at zero, so calls whose work overlaps on the GPU (other
- * streams, other host threads) race: serialise them, e.g. on one stream.
+ * device address (once per device, with the device current) and keeps it for
+ * the life of the process; make that first call before any stream capture, and
+ * do not use this entry point on a device after cudaDeviceReset (the kept
+ * address then names memory of a destroyed context).  Every call shares the
+ * array and clears what must start at zero, so calls whose work overlaps on
+ * the GPU (other streams, other host threads) race: serialise them, e.g. on
+ * one stream.  The kernel's own checks never fault: a block id outside
+ * [0, num_blocks) is read as block 0 and sets PA_DEVERR_BAD_BLOCK, a length
+ * beyond the table sets PA_DEVERR_BAD_LEN, a copy wait that gives up sets
+ * PA_DEVERR_TIMEOUT; those bits collect in the array's error word across calls
+ * until pa_noalloc_check_errors reads them.
  * Errors: PA_ERR_INVALID_ARG (shapes, pointers, lengths; n above 512),
  * PA_ERR_CUDA. */
 pa_status pa_decode_attention_noalloc(const pa_pool_desc *desc, int32_t layer, int32_t n,
                                       const int32_t *block_tables, const int32_t *seq_lens,
                                       int32_t num_q_heads, const void *q, void *out, float scale,
                                       void *stream);
+
+/* The device error bits (PA_DEVERR_*) that pa_decode_attention_noalloc calls
+ * on `device` have set since the last read: synchronises `stream`, reads the
+ * word from the no-allocation scratch array and clears it.  Like the calls it
+ * reports on it allocates nothing, and it shares their array: a read that
+ * overlaps a call on another stream may miss that call's bits, so order it
+ * after the calls it checks.  *bits = 0 before the first call on `device`.
+ * The pages have no counterpart of this call.
+ * Returns PA_ERR_DEVICE_CHECK if any bit was set, PA_ERR_CUDA if a CUDA call
+ * failed, PA_ERR_INVALID_ARG for a null `bits` or a bad ordinal. */
+pa_status pa_noalloc_check_errors(int32_t device, void *stream, uint32_t *bits);
 
 /* Drop `seq`: every block's reference count falls by one, and blocks that
  * reach zero go to the tail of the free list in logical-block order ([MKV]
@@ -276,7 +294,10 @@ pa_status pa_swap_out(pa_pool *pool, int32_t seq, void *host, size_t host_bytes,
  * are private even if the sequence shared blocks before it was swapped out.
  * The new table reaches the device with the next kernel launch on the pool.
  * Errors: PA_ERR_INVALID_ARG, PA_ERR_SEQ_EXISTS, PA_ERR_NO_BLOCKS (checked
- * before any change), PA_ERR_CUDA (the sequence is dropped again). */
+ * before any change; the image and the device are checked before blocks are
+ * taken), PA_ERR_CUDA (a copy could not be enqueued: the sequence is dropped
+ * again and its blocks go back to the free list, but cached blocks that the
+ * reservation evicted stay evicted and the free list's order may differ). */
 pa_status pa_swap_in(pa_pool *pool, int32_t seq, int32_t n_tokens, const void *host,
                      size_t host_bytes, void *stream);
 
@@ -346,7 +367,7 @@ pa_status pa_get_cow_log(pa_pool *pool, int32_t *pairs, int32_t cap, int32_t *n)
 uint64_t pa_launch_count(const pa_pool *pool);
 /* Work plan of the last pa_decode_attention call on this pool:
  * *shared_sets = sibling sets whose common prefix was read once (0 unless
- * partition_tokens was 0), *kv_tiles = (block, KV head) tiles the call reads
+ * partition_tokens was 0), *kv_tiles = (16-token tile, KV head) pairs the call reads
  * from the cache.  Sequences forked from one prompt share the prompt's blocks
  * by reference count ([MKV] Block Tables and Sharing; [PAS] The bonus:
  * sharing via copy-on-write); with partition_tokens = 0 the library reads a
@@ -366,6 +387,22 @@ pa_status pa_last_decode_plan(const pa_pool *pool, int32_t *shared_sets, int64_t
  * PA_ERR_NO_SEQ. */
 pa_status pa_plan_siblings(const pa_pool *pool, int32_t n, const int32_t *seqs, int32_t group,
                            int32_t *set_of, int32_t *set_cp, int32_t *n_sets);
+
+/* Which decode kernel serves a query group of 8 over a 16-bit cache (every
+ * other shape always runs on the warp-level kernel):
+ *   PA_DECODE_WARP    warp-level tensor-core MMAs (mma.sync), 8 workers per SM;
+ *   PA_DECODE_TCGEN05 5th-generation tensor cores: S^T = K Q^T and
+ *                     O^T = V^T P^T accumulate in tensor memory, one worker per
+ *                     SM with 128-token tiles;
+ *   PA_DECODE_AUTO    the library's choice (the faster of the two on B200).
+ * Both compute the same function within the stated tolerance (not bit for
+ * bit).  Errors: PA_ERR_INVALID_ARG. */
+#define PA_DECODE_AUTO 0
+#define PA_DECODE_WARP 1
+#define PA_DECODE_TCGEN05 2
+pa_status pa_set_decode_path(pa_pool *pool, int32_t path);
+/* *tcgen05 = 1 if the last decode call on this pool ran the tcgen05 kernel. */
+pa_status pa_last_decode_kernel(const pa_pool *pool, int32_t *tcgen05);
 
 /* Synchronise `stream`, read the device error word, clear it, and store the
  * PA_DEVERR_* bits in *bits.  Returns PA_ERR_DEVICE_CHECK if any bit was set,

@@ -41,6 +41,7 @@ EXPORTS = (
     "pa_decode_attention_noalloc", "pa_last_decode_plan", "pa_decode_attention_append",
     "pa_plan_siblings", "pa_prefix_register", "pa_prefix_match", "pa_alloc_blocks_prefix",
     "pa_get_cached_blocks", "pa_swap_bytes", "pa_swap_out", "pa_swap_in",
+    "pa_noalloc_check_errors", "pa_set_decode_path", "pa_last_decode_kernel",
 )
 
 
@@ -103,7 +104,13 @@ def lib() -> ctypes.CDLL:
                                                  i32, vp]
         L.pa_decode_attention_noalloc.argtypes = [ctypes.POINTER(pa_pool_desc), i32, i32, vp, _i32p,
                                                   i32, vp, vp, ctypes.c_float, vp]
+        L.pa_noalloc_check_errors.argtypes = [i32, vp, u32p]
+        L.pa_noalloc_check_errors.restype = ctypes.c_int32
         L.pa_free.argtypes = [vp, i32]
+        L.pa_set_decode_path.argtypes = [vp, i32]
+        L.pa_set_decode_path.restype = ctypes.c_int32
+        L.pa_last_decode_kernel.argtypes = [vp, _i32p]
+        L.pa_last_decode_kernel.restype = ctypes.c_int32
         L.pa_prefix_register.argtypes = [vp, i32, i32, _i32p]
         L.pa_prefix_match.argtypes = [vp, i32, _i32p, _i32p]
         L.pa_alloc_blocks_prefix.argtypes = [vp, i32, i32, _i32p, _i32p]
@@ -486,6 +493,33 @@ def pa_check_device_errors(pool: Pool, stream=None) -> int:
     st = lib().pa_check_device_errors(pool.handle, _stream(stream), ctypes.byref(bits))
     if st not in (PA_OK, PA_ERR_DEVICE_CHECK):
         _check(st, "pa_check_device_errors")
+    return bits.value
+
+
+PA_DECODE_AUTO, PA_DECODE_WARP, PA_DECODE_TCGEN05 = 0, 1, 2
+DECODE_PATHS = {"auto": PA_DECODE_AUTO, "warp": PA_DECODE_WARP, "tcgen05": PA_DECODE_TCGEN05}
+
+
+def pa_set_decode_path(pool: Pool, path) -> None:
+    """Kernel for a query group of 8 over 16-bit KV: "auto", "warp" or "tcgen05"."""
+    _check(lib().pa_set_decode_path(pool.handle, DECODE_PATHS.get(path, path)), "pa_set_decode_path")
+
+
+def pa_last_decode_kernel(pool: Pool) -> str:
+    """"tcgen05" if the last decode call ran the tcgen05 kernel, else "warp"."""
+    v = ctypes.c_int32()
+    _check(lib().pa_last_decode_kernel(pool.handle, ctypes.byref(v)), "pa_last_decode_kernel")
+    return "tcgen05" if v.value else "warp"
+
+
+def pa_noalloc_check_errors(device: int = 0, stream=None) -> int:
+    """Synchronise, read and clear the error word of the no-allocation
+    scratch on `device`; returns its bits (raises PAError only for CUDA
+    failures)."""
+    bits = ctypes.c_uint32(0)
+    st = lib().pa_noalloc_check_errors(device, _stream(stream), ctypes.byref(bits))
+    if st not in (PA_OK, PA_ERR_DEVICE_CHECK):
+        _check(st, "pa_noalloc_check_errors")
     return bits.value
 
 

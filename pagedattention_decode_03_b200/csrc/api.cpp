@@ -10,6 +10,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <optional>
 #include <cstring>
 #include <memory>
@@ -109,6 +110,19 @@ struct pa_pool {
   // plan of the last decode call (pa_last_decode_plan)
   int32_t last_sets = 0;
   int64_t last_tiles = 0;
+  int32_t path = PA_DECODE_AUTO;  // pa_set_decode_path
+  bool last_tc = false;
+  // The plan of the last single-launch decode call: the calls of one step
+  // (one per layer) see the same tables, so later ones reuse it.
+  struct PlanCache {
+    bool valid = false, sib = false, tc = false;
+    uint64_t version = 0;
+    int32_t group = 0, mode = 0, part_blocks = 0;
+    int64_t blocks = 0;
+    std::vector<int32_t> seqs;
+    pa::DecodePlan plan;
+    pa::SibPlan sib_plan;
+  } cache;
 };
 
 namespace {
@@ -225,6 +239,9 @@ pa_status bm_status(pa::Status s, const char* what) {
   }
 }
 
+// Which kernel PA_DECODE_AUTO picks for G = 8 over 16-bit KV.
+constexpr bool kAutoTcgen05 = false;
+
 // Shortest common prefix (in full blocks) that is read once for a sibling set.
 constexpr int kMinShareBlocks = 2;
 
@@ -246,7 +263,12 @@ bool build_sib_plan(const pa_pool* p, const int32_t* seqs, int32_t cnt, int grou
   const int max_members = pa::kMaxGroup / group;
   if (max_members < 2 || cnt < 2) return false;
   const pa::BlockManager& bm = *p->bm;
-  auto nb_of = [&](int i) { return (bm.len(seqs[i]) + 15) / 16; };
+  // The kernel walks 16-token tiles (two per 32-token block); sharing is a
+  // property of table entries (blocks), so runs are found in blocks and
+  // placed in tiles.
+  const int tpb = p->d.block_size / 16;
+  auto nb_of = [&](int i) { return (bm.len(seqs[i]) + p->d.block_size - 1) / p->d.block_size; };
+  auto nt_of = [&](int i) { return (bm.len(seqs[i]) + 15) / 16; };
   order.clear();
   for (int i = 0; i < cnt; ++i)
     if (nb_of(i) > kMinShareBlocks) order.push_back(i);
@@ -283,15 +305,16 @@ bool build_sib_plan(const pa_pool* p, const int32_t* seqs, int32_t cnt, int grou
       ++a;
       continue;
     }
-    int64_t pos = cp;
+    const int cpt = cp * tpb;  // shared run in tiles
+    int64_t pos = cpt;
     for (size_t j = a; j < b; ++j) {
       const int it = order[j];
       set_of[it] = nu;
       sp.mem[placed++] = static_cast<int16_t>(it);
       sp.part[it] = static_cast<int32_t>(pos);
-      pos += nb_of(it) - cp;
+      pos += nt_of(it) - cpt;
     }
-    sp.cp[nu] = cp;
+    sp.cp[nu] = cpt;
     work += alpha + pos;
     sp.pre[nu + 1] = static_cast<int32_t>(work);
     sp.mem0[nu + 1] = static_cast<int16_t>(placed);
@@ -307,7 +330,7 @@ bool build_sib_plan(const pa_pool* p, const int32_t* seqs, int32_t cnt, int grou
     sp.mem[placed++] = static_cast<int16_t>(i);
     sp.part[i] = 0;
     sp.cp[nu] = 0;
-    work += alpha + nb_of(i);
+    work += alpha + nt_of(i);
     sp.pre[nu + 1] = static_cast<int32_t>(work);
     sp.mem0[nu + 1] = static_cast<int16_t>(placed);
     ++nu;
@@ -638,6 +661,61 @@ pa_status pa_append_kv(pa_pool* p, int32_t layer, int32_t T, const int32_t* seqs
 
 namespace {
 
+// The plan of one decode launch over the leading items of seqs[0, n): as many
+// as the parameter capacity and (fixed partitions) the workspace's partial
+// slots allow.  *cnt = items taken, *blocks = their 16-token tiles; *sib tells
+// whether a sibling plan (sp) replaces the plain one.
+pa_status plan_launch(pa_pool* p, const int32_t* seqs, int32_t n, int32_t group, int mode,
+                      int32_t part_blocks, int cap, pa::DecodePlan& plan, bool* sib, pa::SibPlan& sp,
+                      int32_t* cnt_out, int64_t* blocks_out) {
+  const int H = p->d.num_kv_heads;
+  const int64_t slots_cap = p->view.partial_slots;
+  const int32_t alpha = pa::stream_k_alpha(p->d.kv_dtype);
+  int32_t cnt = 0;
+  int64_t work = 0, blocks = 0;
+  plan.pre[0] = 0;
+  while (cnt < n && cnt < pa::kDecodeItemsCap) {
+    const int32_t len = p->bm->len(seqs[cnt]);
+    const int32_t nb = (len + 15) / 16;
+    int64_t units = nb + alpha;
+    if (mode == pa::kSplitFixed) units = (nb + part_blocks - 1) / part_blocks;
+    if (mode == pa::kSplitNever) units = 1;
+    if (mode == pa::kSplitFixed && cnt > 0 && (work + units) * H > slots_cap) break;
+    if (cnt > 0 && (work + units) * H >= (int64_t{1} << 30)) break;  // device positions are int32
+    if (mode == pa::kSplitFixed && units * H > slots_cap)
+      return fail(PA_ERR_INVALID_ARG, "partition_tokens too small for the workspace");
+    plan.seq[cnt] = seqs[cnt];
+    plan.len[cnt] = len;
+    work += units;
+    blocks += nb;
+    plan.pre[cnt + 1] = static_cast<int32_t>(work);
+    ++cnt;
+  }
+  plan.n = cnt;
+  plan.mode = mode;
+  plan.part_blocks = part_blocks;
+  plan.alpha = mode == pa::kSplitStreamK ? alpha : 0;
+  plan.pad_ = 0;
+  plan.per_head = work;
+  const int64_t total = work * H;
+  int64_t W = std::min<int64_t>(cap, total);
+  if (mode != pa::kSplitStreamK) {
+    // whole partitions (or sequences) per worker: the same count for every
+    // worker, so no worker runs a round more than the others
+    const int64_t rounds = (total + cap - 1) / cap;
+    W = (total + rounds - 1) / rounds;
+  } else {
+    W = std::min<int64_t>(W, std::max<int64_t>(1, (total + kMinBlocksPerWorker - 1) / kMinBlocksPerWorker));
+    W = std::min<int64_t>(W, slots_cap / 2);
+  }
+  plan.workers = static_cast<int32_t>(std::max<int64_t>(1, W));
+  *sib = mode == pa::kSplitStreamK && group <= 4 &&
+         build_sib_plan(p, seqs, cnt, group, cap, sp, p->order, p->set_of);
+  *cnt_out = cnt;
+  *blocks_out = blocks;
+  return PA_OK;
+}
+
 // pa_decode_attention, and with k_new / v_new the fused append of
 // pa_decode_attention_append (validated by the caller).
 pa_status decode_call(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
@@ -647,8 +725,6 @@ pa_status decode_call(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
   if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
   if (layer < 0 || layer >= p->d.num_layers) return fail(PA_ERR_INVALID_ARG, "layer out of range");
   if (n < 0 || (n > 0 && (!seqs || !q || !out))) return fail(PA_ERR_INVALID_ARG, "null argument");
-  if (p->d.block_size != 16)
-    return fail(PA_ERR_INVALID_ARG, "decode attention supports block_size 16");
   if (num_q_heads <= 0 || num_q_heads % p->d.num_kv_heads != 0)
     return fail(PA_ERR_INVALID_ARG, "num_q_heads must be a multiple of num_kv_heads");
   const int32_t group = num_q_heads / p->d.num_kv_heads;
@@ -665,7 +741,7 @@ pa_status decode_call(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
       return fail(PA_ERR_INVALID_ARG,
                   "partition_tokens must be a multiple of block_size and >= min_partition_tokens");
     mode = pa::kSplitFixed;
-    part_blocks = partition_tokens / p->d.block_size;
+    part_blocks = partition_tokens / 16;  // in the kernel's 16-token tiles
   } else if (partition_tokens != 0) {
     return fail(PA_ERR_INVALID_ARG, "partition_tokens must be 0, -1 or positive");
   }
@@ -688,9 +764,20 @@ pa_status decode_call(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
   if (st != PA_OK) return st;
 
   const int H = p->d.num_kv_heads;
-  const int cap = pa::decode_worker_capacity(p->d.kv_dtype, group, p->num_sms);
-  const int64_t slots_cap = p->view.partial_slots;
+  // G = 8 over 16-bit KV is a real 8-column contraction: the tcgen05 kernel
+  // (one worker per SM) unless the caller asked for the warp-level kernel
+  const bool tc = (p->path == PA_DECODE_TCGEN05 || (p->path == PA_DECODE_AUTO && kAutoTcgen05)) &&
+                  pa::decode_tc_applies(p->d.kv_dtype, group);
+  const int cap = tc ? pa::decode_tc_worker_capacity(p->num_sms)
+                     : pa::decode_worker_capacity(p->d.kv_dtype, group, p->num_sms);
+  p->last_tc = false;
   pa::DecodeArgs args;
+  args.use_tc = 0;
+  static const int l2_ahead = [] {
+    const char* e = std::getenv("PA_L2_AHEAD");
+    return e ? std::atoi(e) : 0;
+  }();
+  args.l2_ahead = l2_ahead;
   args.k_new = k_new;
   args.v_new = v_new;
   args.q = q;
@@ -700,56 +787,42 @@ pa_status decode_call(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
   args.group = group;
   args.scale = scale;
   args.q_item_stride = static_cast<int64_t>(num_q_heads) * pa::kHeadDim;
-  static thread_local pa::DecodePlan plan;
-  const int32_t alpha = pa::stream_k_alpha(p->d.kv_dtype);
+  pa_pool::PlanCache& pc = p->cache;
+  const bool hit = pc.valid && pc.version == p->bm->version() && pc.group == group && pc.mode == mode &&
+                   pc.part_blocks == part_blocks && pc.tc == tc &&
+                   pc.seqs.size() == static_cast<size_t>(n) &&
+                   std::equal(seqs, seqs + n, pc.seqs.begin());
+  pa::DecodePlan& plan = pc.plan;
   int32_t at = 0;
   while (at < n) {
     // Items of this launch: up to the parameter capacity, and (fixed mode) the
     // partial slots the workspace holds.
     int32_t cnt = 0;
-    int64_t work = 0, blocks = 0;
-    plan.pre[0] = 0;
-    while (at + cnt < n && cnt < pa::kDecodeItemsCap) {
-      const int32_t len = p->bm->len(seqs[at + cnt]);
-      const int32_t nb = (len + 15) / 16;
-      int64_t units = nb + alpha;
-      if (mode == pa::kSplitFixed) units = (nb + part_blocks - 1) / part_blocks;
-      if (mode == pa::kSplitNever) units = 1;
-      if (mode == pa::kSplitFixed && cnt > 0 && (work + units) * H > slots_cap) break;
-      if (cnt > 0 && (work + units) * H >= (int64_t{1} << 30)) break;  // device positions are int32
-      if (mode == pa::kSplitFixed && units * H > slots_cap)
-        return fail(PA_ERR_INVALID_ARG, "partition_tokens too small for the workspace");
-      plan.seq[cnt] = seqs[at + cnt];
-      plan.len[cnt] = len;
-      work += units;
-      blocks += nb;
-      plan.pre[cnt + 1] = static_cast<int32_t>(work);
-      ++cnt;
-    }
-    plan.n = cnt;
-    plan.mode = mode;
-    plan.part_blocks = part_blocks;
-    plan.alpha = mode == pa::kSplitStreamK ? alpha : 0;
-    plan.pad_ = 0;
-    plan.per_head = work;
-    const int64_t total = work * H;
-    int64_t W = std::min<int64_t>(cap, total);
-    if (mode != pa::kSplitStreamK) {
-      // whole partitions (or sequences) per worker: the same count for every
-      // worker, so no worker runs a round more than the others
-      const int64_t rounds = (total + cap - 1) / cap;
-      W = (total + rounds - 1) / rounds;
+    int64_t blocks = 0;
+    if (hit) {  // the previous call's single launch, same tables
+      cnt = n;
+      blocks = pc.blocks;
     } else {
-      W = std::min<int64_t>(W, std::max<int64_t>(1, (total + kMinBlocksPerWorker - 1) / kMinBlocksPerWorker));
-      W = std::min<int64_t>(W, slots_cap / 2);
+      pc.valid = false;
+      const pa_status st = plan_launch(p, seqs + at, n - at, group, mode, part_blocks, cap, plan,
+                                       &pc.sib, pc.sib_plan, &cnt, &blocks);
+      if (st != PA_OK) return st;
+      if (at == 0 && cnt == n) {
+        pc.valid = true;
+        pc.version = p->bm->version();
+        pc.group = group;
+        pc.mode = mode;
+        pc.part_blocks = part_blocks;
+        pc.tc = tc;
+        pc.blocks = blocks;
+        pc.seqs.assign(seqs, seqs + n);
+      }
     }
-    plan.workers = static_cast<int32_t>(std::max<int64_t>(1, W));
     args.item_offset = at;
     int launches = 0;
     cudaError_t e;
-    static thread_local pa::SibPlan sib;
-    if (mode == pa::kSplitStreamK && group <= 4 &&
-        build_sib_plan(p, seqs + at, cnt, group, cap, sib, p->order, p->set_of)) {
+    const pa::SibPlan& sib = pc.sib_plan;
+    if (pc.sib) {
       if (k_new != nullptr) {
         // Sibling sets put several sequences' last blocks back to back in one
         // worker's share; that worker's row patches would run in series, so the
@@ -772,8 +845,11 @@ pa_status decode_call(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
       p->last_sets += sib.sets;
       p->last_tiles += (sib.per_head - static_cast<int64_t>(sib.alpha) * sib.nu) * H;
     } else {
+      args.use_tc = tc ? 1 : 0;
       e = pa::launch_decode(p->view, &p->tmk, &p->tmv, plan, args, s, &launches);
+      args.use_tc = 0;
       p->last_tiles += blocks * H;
+      p->last_tc = p->last_tc || tc;
     }
     p->launches += launches;
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
@@ -883,6 +959,22 @@ pa_status pa_get_cow_log(pa_pool* p, int32_t* pairs, int32_t cap, int32_t* n) {
 
 uint64_t pa_launch_count(const pa_pool* p) { return p ? p->launches : 0; }
 
+pa_status pa_set_decode_path(pa_pool* p, int32_t path) {
+  g_last_error.clear();
+  if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
+  if (path != PA_DECODE_AUTO && path != PA_DECODE_WARP && path != PA_DECODE_TCGEN05)
+    return fail(PA_ERR_INVALID_ARG, "path must be PA_DECODE_AUTO, PA_DECODE_WARP or PA_DECODE_TCGEN05");
+  p->path = path;
+  return PA_OK;
+}
+
+pa_status pa_last_decode_kernel(const pa_pool* p, int32_t* tcgen05) {
+  g_last_error.clear();
+  if (!p || !tcgen05) return fail(PA_ERR_INVALID_ARG, "null argument");
+  *tcgen05 = p->last_tc ? 1 : 0;
+  return PA_OK;
+}
+
 pa_status pa_plan_siblings(const pa_pool* p, int32_t n, const int32_t* seqs, int32_t group,
                            int32_t* set_of, int32_t* set_cp, int32_t* n_sets) {
   g_last_error.clear();
@@ -903,7 +995,8 @@ pa_status pa_plan_siblings(const pa_pool* p, int32_t n, const int32_t* seqs, int
   int32_t sets = 0;
   if (build_sib_plan(p, seqs, n, group, pa::kMaxWorkers, sp, order, set_idx)) sets = sp.sets;
   for (int32_t i = 0; i < n; ++i) set_of[i] = sets ? set_idx[i] : -1;
-  for (int32_t k = 0; k < sets; ++k) set_cp[k] = sp.cp[k];
+  const int tpb = p->d.block_size / 16;  // the plan counts 16-token tiles
+  for (int32_t k = 0; k < sets; ++k) set_cp[k] = sp.cp[k] / tpb;
   *n_sets = sets;
   return PA_OK;
 }

@@ -179,10 +179,12 @@ void BlockManager::unregister(int32_t block) {
 
 void BlockManager::record_entry(int32_t seq, int32_t j, int32_t block) {
   deltas_.set(static_cast<int64_t>(seq) * mbps_ + j, block);
+  ++version_;
 }
 
 void BlockManager::record_len(int32_t seq, int32_t len) {
   deltas_.set(static_cast<int64_t>(max_seqs_) * mbps_ + seq, len);
+  ++version_;
 }
 
 Status BlockManager::reserve(int32_t seq, int32_t new_len, std::vector<CowPair>* cows) {

@@ -140,12 +140,16 @@ class BlockManager {
   void set_fail_after(int64_t n) { fail_after_ = n; }
   MirrorDeltas& deltas() { return deltas_; }
 
+  // Incremented by every change of a block table or a length: equal versions
+  // mean identical tables (a decode plan built from them is still valid).
+  uint64_t version() const { return version_; }
   int32_t num_blocks() const { return num_blocks_; }
   int32_t block_size() const { return block_size_; }
   int32_t max_seqs() const { return max_seqs_; }
   int32_t max_blocks_per_seq() const { return mbps_; }
 
  private:
+  uint64_t version_ = 0;
   struct Seq {
     bool active = false;
     int32_t len = 0;

@@ -54,9 +54,8 @@ namespace pa {
 namespace {
 
 constexpr int kWarps = 4;              // warps (independent workers) per CTA
-constexpr int kBlock = 16;             // tokens per KV block handled by the kernel
-constexpr uint32_t kWaitLimit = 1u << 22;
-constexpr float kLog2e = 1.4426950408889634f;
+
+#include "decode_common.cuh"
 
 template <int KV>
 struct Tile {
@@ -65,299 +64,6 @@ struct Tile {
   static constexpr int kStages = KV == kFP8 ? 6 : 3;
   static constexpr int kRingBytes = kStages * kStageBytes;
 };
-
-template <class PlanT>
-struct DecodeKParams {
-  const uint8_t* q;
-  uint8_t* out;
-  const int32_t* tables;
-  float* partials;
-  int32_t* counters;       // stream-K arrival counters (zero between launches)
-  uint32_t* err;
-  const float* k_scale;
-  const float* v_scale;
-  int64_t q_item_stride;   // elements between items of q / out
-  float scale;
-  int32_t layer, num_kv_heads, num_blocks, mbps, group;
-  int64_t total;           // work units over all heads
-  // Fused append (null k_new: none): the K/V rows of each item's last token,
-  // [n][H][128] act dtype, written into the cache by the worker that reads the
-  // item's last block, which also patches them into its staged tile.
-  const uint8_t* k_new;
-  const uint8_t* v_new;
-  uint8_t* k_cache;
-  uint8_t* v_cache;
-  const float* k_inv;
-  const float* v_inv;
-  PlanT plan;
-};
-
-template <class PlanT>
-constexpr bool kIsSib = std::is_same<PlanT, SibPlan>::value;
-template <class Prm>
-constexpr bool kSibParams = std::is_same<Prm, DecodeKParams<SibPlan>>::value;
-
-// A worker's contiguous piece of one work unit.  Positions b0 .. b1-1 are the
-// unit's KV blocks in order (for a plain unit: table blocks of item i).
-struct Seg {
-  int32_t h, i, b0, b1, dest, len, seq;
-  int32_t k;      // work unit (== i for plain plans)
-  bool valid;
-  bool shared;    // a sibling set (two or more items) of a sibling plan
-};
-
-// Table position, valid length and active query rows of one KV block.
-struct BlockRef {
-  int32_t seq, b, len;
-  uint32_t cols;  // bit r set: query row r takes part (all 8 for plain units)
-  int32_t item;   // the item whose table row this is
-};
-
-__device__ __forceinline__ int n_entries(const DecodePlan& P) { return P.n; }
-__device__ __forceinline__ int n_entries(const SibPlan& P) { return P.nu; }
-__device__ __forceinline__ int plan_mode(const DecodePlan& P) { return P.mode; }
-__device__ __forceinline__ int plan_mode(const SibPlan&) { return kSplitStreamK; }
-
-// Index of the entry whose prefix range holds r: pre[i] <= r < pre[i+1].
-template <class PlanT>
-__device__ __forceinline__ int find_item(const PlanT& P, int64_t r) {
-  int lo = 0, hi = n_entries(P) - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (P.pre[mid] <= r) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
-// find_item, first trying `hint` and the entry after it (a worker's next
-// segment almost always starts in one of those).
-template <class PlanT>
-__device__ __forceinline__ int find_item_hint(const PlanT& P, int64_t r, int hint) {
-  const int n = n_entries(P);
-  if (hint >= 0 && hint < n && P.pre[hint] <= r) {
-    if (r < P.pre[hint + 1]) return hint;
-    if (hint + 1 < n && r < P.pre[hint + 2]) return hint + 1;
-  }
-  return find_item(P, r);
-}
-
-__device__ __forceinline__ int64_t worker_start(int64_t total, int w, int W) {
-  return (total * w) / W;
-}
-
-// Worker whose share [worker_start(w), worker_start(w+1)) holds position x:
-// the largest w with total*w < (x+1)*W.
-__device__ __forceinline__ int find_worker(int64_t total, int W, int64_t x) {
-  return min(W - 1, static_cast<int>(((x + 1) * W - 1) / total));
-}
-
-// Stream-K piece of one unit.  A unit occupies alpha + nb positions of the
-// work axis: alpha positions that stand for the fixed cost of a segment
-// (begin, finish, partial write and arrival) and carry no block, then its nb
-// KV blocks.  Shares are equal in positions, so a worker whose share crosses
-// unit boundaries gets fewer blocks.  From position r (offset o = r - v0 in
-// the unit [v0, v1)) the worker takes `take` positions; the piece reads blocks
-// [b0, b1).  Returns false when those positions hold no block.  A piece that
-// covers the unit's blocks only in part writes partial slot 2w if it starts
-// inside the blocks (it holds the share's start; one per worker), else 2w+1
-// (it holds the share's end).
-__device__ __forceinline__ bool stream_piece(int64_t r, int32_t v0, int32_t v1, int32_t alpha,
-                                             int64_t avail, int w, int64_t& take, Seg& s) {
-  const int32_t unit_nb = v1 - v0 - alpha;
-  take = min(static_cast<int64_t>(v1) - r, avail);
-  const int64_t o = r - v0;
-  s.b0 = static_cast<int32_t>(max(o - alpha, int64_t{0}));
-  s.b1 = static_cast<int32_t>(max(o + take - alpha, int64_t{0}));
-  if (s.b1 <= s.b0) return false;
-  const bool whole = s.b0 == 0 && s.b1 == unit_nb;
-  s.dest = whole ? -1 : (s.b0 > 0 ? 2 * w : 2 * w + 1);
-  return true;
-}
-
-// Next segment of worker `w` within the remaining range [g, g_end) of its
-// share; `hint` carries the entry of the previous segment.
-__device__ __forceinline__ Seg next_seg(const DecodeKParams<DecodePlan>& prm, int64_t& g,
-                                        int64_t g_end, int w, int64_t /*g0*/, int& hint) {
-  Seg s;
-  s.shared = false;
-  const DecodePlan& P = prm.plan;
-  const int64_t per_head = P.per_head;
-  for (;;) {
-    s.valid = g < g_end;
-    if (!s.valid) return s;
-    s.h = static_cast<int32_t>(g / per_head);
-    const int64_t r = g - static_cast<int64_t>(s.h) * per_head;
-    if (P.mode == kSplitNever) {
-      s.i = static_cast<int32_t>(r);
-    } else {
-      s.i = find_item_hint(P, r, hint);
-      hint = s.i;
-    }
-    s.k = s.i;
-    s.seq = P.seq[s.i];
-    s.len = P.len[s.i];
-    int32_t nb = (s.len + kBlock - 1) / kBlock;
-    if (s.len <= 0 || nb > prm.mbps) {
-      atomicOr(prm.err, kErrBadLen);
-      nb = min(max(nb, 1), prm.mbps);
-      s.len = max(s.len, 1);
-    }
-    if (P.mode == kSplitStreamK) {
-      const int32_t v0 = P.pre[s.i], v1 = P.pre[s.i + 1];
-      if (v1 - v0 - P.alpha != nb) atomicOr(prm.err, kErrBadLen);
-      int64_t take;
-      const bool any = stream_piece(r, v0, v1, P.alpha, g_end - g, w, take, s);
-      g += take;
-      if (!any) continue;
-    } else if (P.mode == kSplitFixed) {
-      const int32_t p = static_cast<int32_t>(r - P.pre[s.i]);
-      const int32_t np = P.pre[s.i + 1] - P.pre[s.i];
-      s.b0 = p * P.part_blocks;
-      s.b1 = min(nb, s.b0 + P.part_blocks);
-      if (s.b0 >= s.b1) {  // inconsistent lengths: clamp to an empty-free range
-        atomicOr(prm.err, kErrBadLen);
-        s.b0 = max(0, s.b1 - 1);
-      }
-      s.dest = np == 1 ? -1 : static_cast<int32_t>(g);
-      g += 1;
-    } else {
-      s.b0 = 0;
-      s.b1 = nb;
-      s.dest = -1;
-      g += 1;
-    }
-    return s;
-  }
-}
-
-// Sibling plan (always stream-K): same cutting and partial slots as a plain
-// stream-K plan, over units that may hold several items.
-__device__ __forceinline__ Seg next_seg(const DecodeKParams<SibPlan>& prm, int64_t& g,
-                                        int64_t g_end, int w, int64_t /*g0*/, int& hint) {
-  Seg s;
-  const SibPlan& P = prm.plan;
-  for (;;) {
-    s.valid = g < g_end;
-    if (!s.valid) return s;
-    s.h = static_cast<int32_t>(g / P.per_head);
-    const int64_t r = g - static_cast<int64_t>(s.h) * P.per_head;
-    s.k = find_item_hint(P, r, hint);
-    hint = s.k;
-    const int m0 = P.mem0[s.k];
-    s.shared = P.mem0[s.k + 1] - m0 > 1;
-    s.i = P.mem[m0];
-    s.seq = P.seq[s.i];
-    s.len = P.len[s.i];
-    const int32_t v0 = P.pre[s.k], v1 = P.pre[s.k + 1];
-    const int32_t unit_nb = v1 - v0 - P.alpha;
-    if (!s.shared && (s.len <= 0 || (s.len + kBlock - 1) / kBlock != unit_nb || unit_nb > prm.mbps))
-      atomicOr(prm.err, kErrBadLen);
-    int64_t take;
-    const bool any = stream_piece(r, v0, v1, P.alpha, g_end - g, w, take, s);
-    g += take;
-    if (any) return s;
-  }
-}
-
-// Where position o of segment s lives.  Plain plans: block o of the item.
-// Sibling plans: positions below the unit's shared run cp are the common
-// blocks (every row takes part); after it come the members' own blocks in
-// member order, each taken only by that member's G rows.
-template <int G>
-__device__ __forceinline__ BlockRef locate(const DecodeKParams<DecodePlan>&, const Seg& s, int o) {
-  return BlockRef{s.seq, o, s.len, 0xffu, s.i};
-}
-template <int G>
-__device__ __forceinline__ BlockRef locate(const DecodeKParams<SibPlan>& prm, const Seg& s, int o) {
-  const SibPlan& P = prm.plan;
-  const int cp = P.cp[s.k];
-  if (o < cp) return BlockRef{s.seq, o, s.len, 0xffu, s.i};
-  const int m0 = P.mem0[s.k], m = P.mem0[s.k + 1] - m0;
-  int j = 0, item = s.i;
-  for (int jj = 1; jj < m; ++jj) {
-    const int it = P.mem[m0 + jj];
-    if (P.part[it] > o) break;
-    j = jj;
-    item = it;
-  }
-  return BlockRef{P.seq[item], cp + (o - P.part[item]), P.len[item],
-                  ((1u << G) - 1u) << (j * G), item};
-}
-
-// The segments of one worker, in processing order.  Stream-K: a worker's last
-// segment, when it starts inside the worker's share (the head of a sequence
-// cut at the share's end), is processed first, then the share from its start
-// (whose first segment is the tail of a sequence cut at the share's start).
-// Both halves of every cut sequence thus finish early and the merge of their
-// partial results happens off the kernel's critical path.
-struct Cursor {
-  int64_t g, end, g0, glast;
-  int w;
-  int hint, hint_g0;  // entry of the next segment, and of the share's start
-  bool second;
-
-  template <class Prm>
-  __device__ __forceinline__ void init(const Prm& prm, int64_t s0, int64_t s1, int wk) {
-    g0 = s0;
-    w = wk;
-    glast = s0;
-    hint = hint_g0 = -1;
-    const auto& P = prm.plan;
-    if (plan_mode(P) == kSplitStreamK && s1 > s0) {
-      // entries of the share's last and first positions, two searches
-      // interleaved so their dependent loads overlap
-      const int64_t x = s1 - 1;
-      const int64_t h = x / P.per_head;
-      const int64_t r1 = x - h * P.per_head;
-      const int64_t r0 = s0 - (s0 / P.per_head) * P.per_head;
-      int lo1 = 0, hi1 = n_entries(P) - 1, lo0 = 0, hi0 = hi1;
-      while (lo1 < hi1 || lo0 < hi0) {
-        if (lo1 < hi1) {
-          const int mid = (lo1 + hi1 + 1) >> 1;
-          if (P.pre[mid] <= r1) lo1 = mid; else hi1 = mid - 1;
-        }
-        if (lo0 < hi0) {
-          const int mid = (lo0 + hi0 + 1) >> 1;
-          if (P.pre[mid] <= r0) lo0 = mid; else hi0 = mid - 1;
-        }
-      }
-      glast = max(s0, h * P.per_head + P.pre[lo1]);
-      hint = lo1;
-      hint_g0 = lo0;
-    }
-    g = glast;
-    end = s1;
-    second = false;
-  }
-
-  template <class Prm>
-  __device__ __forceinline__ Seg next(const Prm& prm) {
-    for (;;) {
-      if (g >= end && !second && glast > g0) {
-        second = true;
-        g = g0;
-        end = glast;
-        hint = hint_g0;
-      }
-      const Seg s = next_seg(prm, g, end, w, g0, hint);
-      // the first phase may hold only cost positions: go on with the second
-      if (s.valid || second || glast <= g0) return s;
-    }
-  }
-};
-
-// ------------------------------------------------------ fused append rows
-__device__ __forceinline__ bool is_last_block(const BlockRef& br) { return br.b == (br.len - 1) / kBlock; }
-
-// Address of this lane's 16 bytes of the rows.  (Calls whose plan has sibling
-// sets append with the append kernel instead: a set puts several sequences'
-// last blocks into one worker's share, and their row loads would run in
-// series.)
-template <class Prm>
-__device__ __forceinline__ const uint4* new_row_ptr(const Prm& prm, int h, int item, int lane) {
-  const int64_t src_el = (static_cast<int64_t>(item) * prm.num_kv_heads + h) * kHeadDim + (lane & 15) * 8;
-  return reinterpret_cast<const uint4*>((lane < 16 ? prm.k_new : prm.v_new) + src_el * 2);
-}
 
 
 // ------------------------------------------------------------------ producer
@@ -368,7 +74,7 @@ struct Producer {
   int32_t b;          // next block of seg to fetch
   int32_t tc_val, tc_base, tc_unit;
   uint32_t issued;
-  int32_t* phys_s;    // shared memory: physical block id of each stage
+  int32_t* phys_s;    // shared memory: first cache row (token slot) of each staged tile
 
   // Starts from a copy of the consumer's cursor (same segments, same order).
   template <class Prm>
@@ -393,25 +99,32 @@ struct Producer {
       if (!seg.valid) return;
       b = seg.b0;
     }
-    // physical ids of the unit's positions b .. b+31, one per lane (a sibling
-    // set's positions run through several table rows)
+    // physical ids of the unit's tiles b .. b+31, one per lane (a sibling
+    // set's positions run through several table rows); the low bit of a
+    // 32-token block's tile index picks its half
     if (seg.k != tc_unit || b < tc_base || b >= tc_base + 32) {
       tc_unit = seg.k;
       tc_base = b;
       const BlockRef r = locate<1>(prm, seg, b + lane);
-      tc_val = r.b >= 0 && r.b < prm.mbps ? prm.tables[static_cast<int64_t>(r.seq) * prm.mbps + r.b] : 0;
+      const int32_t e = r.b >> prm.bshift;
+      tc_val = r.b >= 0 && e < prm.mbps ? prm.tables[static_cast<int64_t>(r.seq) * prm.mbps + e] : 0;
+      // physical id in the upper bits, half in bit 0 (ids < 2^30)
+      tc_val = static_cast<int32_t>((static_cast<uint32_t>(tc_val) << 1) |
+                                    static_cast<uint32_t>(r.b & ((1 << prm.bshift) - 1)));
     }
-    int32_t phys = __shfl_sync(0xffffffffu, tc_val, b - tc_base);
+    const int32_t tv = __shfl_sync(0xffffffffu, tc_val, b - tc_base);
+    int32_t phys = static_cast<int32_t>(static_cast<uint32_t>(tv) >> 1);
     if (static_cast<uint32_t>(phys) >= static_cast<uint32_t>(prm.num_blocks)) {
       if (lane == 0) atomicOr(prm.err, kErrBadBlock);
       phys = 0;
     }
     const uint32_t stage = issued % Tile<KV>::kStages;
     const uint32_t bar = bars + stage * 8;
-    if (lane == 0) phys_s[stage] = phys;
     const uint32_t dst = ring + stage * Tile<KV>::kStageBytes;
     const int32_t row =
-        ((prm.layer * prm.num_blocks + phys) * prm.num_kv_heads + seg.h) * kBlock;
+        (((prm.layer * prm.num_blocks + phys) * prm.num_kv_heads + seg.h) << (4 + prm.bshift)) +
+        (tv & 1) * kBlock;
+    if (lane == 0) phys_s[stage] = row;
     if (lane == 0) {
       dev::mbar_arrive_expect_tx(bar, Tile<KV>::kStageBytes);
       if constexpr (KV == kFP8) {
@@ -422,6 +135,24 @@ struct Producer {
         dev::tma_load_2d(dst + 2048, tmk, 64, row, bar);
         dev::tma_load_2d(dst + Tile<KV>::kBytes, tmv, 0, row, bar);
         dev::tma_load_2d(dst + Tile<KV>::kBytes + 2048, tmv, 64, row, bar);
+      }
+    }
+    // The tile l2_ahead positions further on goes to L2 now, so more of the
+    // worker's reads are in flight than its shared-memory ring holds.
+    const int32_t pb = b + prm.l2_ahead;
+    if (prm.l2_ahead > 0 && pb < seg.b1 && pb - tc_base < 32) {
+      const int32_t pv = __shfl_sync(0xffffffffu, tc_val, pb - tc_base);
+      const int32_t pphys = static_cast<int32_t>(static_cast<uint32_t>(pv) >> 1);
+      if (lane == 0 && static_cast<uint32_t>(pphys) < static_cast<uint32_t>(prm.num_blocks)) {
+        const int32_t prow =
+            (((prm.layer * prm.num_blocks + pphys) * prm.num_kv_heads + seg.h) << (4 + prm.bshift)) +
+            (pv & 1) * kBlock;
+        dev::tma_prefetch_l2_2d(tmk, 0, prow);
+        dev::tma_prefetch_l2_2d(tmv, 0, prow);
+        if constexpr (KV != kFP8) {
+          dev::tma_prefetch_l2_2d(tmk, 64, prow);
+          dev::tma_prefetch_l2_2d(tmv, 64, prow);
+        }
       }
     }
     ++issued;
@@ -448,224 +179,6 @@ __device__ __forceinline__ void zero_tail_rows(uint8_t* vtile, int nvalid, int l
   }
   dev::fence_proxy_async_smem();
   __syncwarp();
-}
-
-__device__ __forceinline__ float warp_max_rows(float x) {  // over lanes sharing lane & 3
-  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
-  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
-  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
-  return x;
-}
-__device__ __forceinline__ float warp_sum_rows(float x) {
-  x += __shfl_xor_sync(0xffffffffu, x, 4);
-  x += __shfl_xor_sync(0xffffffffu, x, 8);
-  x += __shfl_xor_sync(0xffffffffu, x, 16);
-  return x;
-}
-
-template <int ACT>
-__device__ __forceinline__ float act_to_f32(uint16_t x) {
-  if constexpr (ACT == kBF16) return __uint_as_float(static_cast<uint32_t>(x) << 16);
-  else return __half2float(__ushort_as_half(x));
-}
-
-template <int ACT>
-__device__ __forceinline__ uint16_t f32_to_act(float x) {
-  if constexpr (ACT == kBF16) return __bfloat16_as_ushort(__float2bfloat16_rn(x));
-  else return __half_as_ushort(__float2half_rn(x));
-}
-
-// ================================================================ LSE merge
-// One warp's share of a log-sum-exp merge: query row `gg` over partial slots
-// kb .. ke-1, each (m, l, o~).  Leaves M = max m_k, L = sum 2^(m_k - M) l_k and
-// acc = sum 2^(m_k - M) o~_k (d = 4*lane .. 4*lane+3), unnormalised; M = -inf
-// for an empty range.  Partials written by other SMs are read through L2
-// (ld.global.cg): the (m, l) pairs 32 slots at a time across the lanes, the o~
-// rows 32 slots at a time with every load issued before any use.
-template <class SlotFn>
-__device__ __forceinline__ void merge_row_part(const float* partials, int gg, int kb, int ke,
-                                               SlotFn slot_of, int lane, float& M, float& L,
-                                               float4& acc) {
-  auto ml_of = [&](int k) {
-    return partials + static_cast<int64_t>(slot_of(k)) * kPartialSlotFloats + kMaxGroup * kHeadDim +
-           2 * gg;
-  };
-  M = -INFINITY;
-  for (int k = kb + lane; k < ke; k += 32) M = fmaxf(M, __ldcg(ml_of(k)));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float ref = M == -INFINITY ? 0.f : M;
-  constexpr int kInFlight = 32;
-  L = 0.f;
-  acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int k0 = kb; k0 < ke; k0 += kInFlight) {
-    const int k = k0 + lane;
-    float wk = 0.f;
-    if (k < ke) {
-      const float2 ml = __ldcg(reinterpret_cast<const float2*>(ml_of(k)));
-      wk = dev::exp2_approx(ml.x - ref);
-      L += wk * ml.y;
-    }
-    const int cnt = min(kInFlight, ke - k0);
-    float4 x[kInFlight];
-#pragma unroll
-    for (int t = 0; t < kInFlight; ++t) {
-      if (t < cnt)
-        x[t] = __ldcg(reinterpret_cast<const float4*>(
-                          partials + static_cast<int64_t>(slot_of(k0 + t)) * kPartialSlotFloats +
-                          gg * kHeadDim) + lane);
-    }
-#pragma unroll
-    for (int t = 0; t < kInFlight; ++t) {
-      const float wj = __shfl_sync(0xffffffffu, wk, t);
-      if (t < cnt) {
-        acc.x += wj * x[t].x;
-        acc.y += wj * x[t].y;
-        acc.z += wj * x[t].z;
-        acc.w += wj * x[t].w;
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-}
-
-// Query rows of a segment: a plain unit has its item's G query heads of KV
-// head h (rows 0 .. G-1); a sibling set has member j's G heads at rows
-// j*G .. j*G+G-1.  item_of_row(r) is the item whose output row r is.
-template <int G>
-__device__ __forceinline__ int unit_rows(const DecodeKParams<DecodePlan>&, const Seg&) { return G; }
-template <int G>
-__device__ __forceinline__ int unit_rows(const DecodeKParams<SibPlan>& prm, const Seg& s) {
-  return (prm.plan.mem0[s.k + 1] - prm.plan.mem0[s.k]) * G;
-}
-template <int G>
-__device__ __forceinline__ int item_of_row(const DecodeKParams<DecodePlan>&, const Seg& s, int) {
-  return s.i;
-}
-template <int G>
-__device__ __forceinline__ int item_of_row(const DecodeKParams<SibPlan>& prm, const Seg& s, int r) {
-  return prm.plan.mem[prm.plan.mem0[s.k] + r / G];
-}
-// Element offset of (row r, d = 0) in q / out.
-template <int G, class Prm>
-__device__ __forceinline__ int64_t row_offset(const Prm& prm, const Seg& s, int r) {
-  return item_of_row<G>(prm, s, r) * prm.q_item_stride + (s.h * G + r % G) * kHeadDim;
-}
-
-// One warp merges query rows 0 .. rows-1 (rows <= R) of one unit over
-// `nslots` partial slots, online: for each slot k (m_k, l_k, o~_k) the running
-// (M, L, acc) become
-//   M' = max(M, m_k), L' = L 2^(M-M') + l_k 2^(m_k-M'), acc' likewise,
-// with 0 in place of M' while every slot seen so far is empty (m = -inf, a
-// row that no token of those slots reached).
-// Slots are taken a few at a time with every load of a batch issued before
-// any use, so a typical cut sequence (2-4 partials) costs one L2 round trip.
-// Each lane owns d = 4*lane .. 4*lane+3 of every row and reads the (m, l)
-// pairs itself (same address in all lanes: one broadcast transaction).
-// out_of(r) = element offset of output row r.
-template <int ACT, int R, class SlotFn, class OutFn>
-__device__ __forceinline__ void merge_unit_warp(const float* partials, uint16_t* out, int nslots,
-                                                int rows, SlotFn slot_of, OutFn out_of, int lane) {
-  constexpr int kBatch = R >= 8 ? 2 : (R >= 4 ? 3 : 4);  // loads in flight within the register budget
-  float M[R], L[R];
-  float4 acc[R];
-#pragma unroll
-  for (int gg = 0; gg < R; ++gg) {
-    M[gg] = -INFINITY;
-    L[gg] = 0.f;
-    acc[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  for (int k0 = 0; k0 < nslots; k0 += kBatch) {
-    float2 ml[kBatch][R];
-    float4 x[kBatch][R];
-#pragma unroll
-    for (int j = 0; j < kBatch; ++j) {
-      if (k0 + j < nslots) {
-        const float* slot = partials + static_cast<int64_t>(slot_of(k0 + j)) * kPartialSlotFloats;
-#pragma unroll
-        for (int gg = 0; gg < R; ++gg) {
-          if (gg < rows) {
-            ml[j][gg] = __ldcg(reinterpret_cast<const float2*>(slot + kMaxGroup * kHeadDim) + gg);
-            x[j][gg] = __ldcg(reinterpret_cast<const float4*>(slot + gg * kHeadDim) + lane);
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kBatch; ++j) {
-      if (k0 + j < nslots) {
-#pragma unroll
-        for (int gg = 0; gg < R; ++gg) {
-          if (gg < rows) {
-            const float mn = fmaxf(M[gg], ml[j][gg].x);
-            const float ref = mn == -INFINITY ? 0.f : mn;
-            const float a = dev::exp2_approx(M[gg] - ref);        // 0 on the first slot
-            const float b = dev::exp2_approx(ml[j][gg].x - ref);
-            M[gg] = mn;
-            L[gg] = L[gg] * a + ml[j][gg].y * b;
-            acc[gg].x = acc[gg].x * a + x[j][gg].x * b;
-            acc[gg].y = acc[gg].y * a + x[j][gg].y * b;
-            acc[gg].z = acc[gg].z * a + x[j][gg].z * b;
-            acc[gg].w = acc[gg].w * a + x[j][gg].w * b;
-          }
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int gg = 0; gg < R; ++gg) {
-    if (gg < rows) {
-      const float inv = 1.f / L[gg];
-      const uint32_t a = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].x * inv)) |
-                         (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].y * inv)) << 16);
-      const uint32_t b = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].z * inv)) |
-                         (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].w * inv)) << 16);
-      *reinterpret_cast<uint2*>(out + out_of(gg) + 4 * lane) = make_uint2(a, b);
-    }
-  }
-}
-
-__device__ __forceinline__ int atom_add_acq_rel(int32_t* p, int32_t v) {
-  int32_t old;
-  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-
-// Stream-K: after a worker wrote the partial of a cut unit, it counts itself
-// in; the last of the unit's workers merges all of them into the output and
-// re-arms the counter.  (Counter = the unit's first worker, unique per cut
-// unit.)  R = row capacity of the merge (rows <= R).
-template <int ACT, int G, int R, class Prm>
-__device__ __forceinline__ void settle_partial(const Prm& prm, const Seg& s, int rows, int lane) {
-  const auto& P = prm.plan;
-  if (plan_mode(P) != kSplitStreamK) return;  // fixed partitions: a separate reduce kernel merges
-  const int W = P.workers;
-  // the unit's blocks: positions [u0, u1) (after its alpha cost positions)
-  const int64_t u0 = static_cast<int64_t>(s.h) * P.per_head + P.pre[s.k] + P.alpha;
-  const int64_t u1 = static_cast<int64_t>(s.h) * P.per_head + P.pre[s.k + 1];
-  const int wa = find_worker(prm.total, W, u0);
-  const int wb = find_worker(prm.total, W, u1 - 1);
-  const int nslots = wb - wa + 1;
-  // __syncwarp orders the other lanes' partial writes before lane 0's
-  // release; the acquire half orders the merge's reads after the arrivals.
-  __syncwarp();
-  int old = 0;
-  if (lane == 0) old = atom_add_acq_rel(prm.counters + wa, 1);
-  old = __shfl_sync(0xffffffffu, old, 0);
-  if (old != nslots - 1) return;
-  __syncwarp();
-  // wa's piece starts inside the blocks (slot 2wa) only if its share does
-  const bool a_inside = worker_start(prm.total, wa, W) > u0;
-  auto slot_of = [&](int q) {
-    const int wk = wa + q;
-    return (q == 0 && !a_inside) ? 2 * wk + 1 : 2 * wk;
-  };
-  auto out_of = [&](int r) { return row_offset<G>(prm, s, r); };
-  uint16_t* out = reinterpret_cast<uint16_t*>(prm.out);
-  merge_unit_warp<ACT, R>(prm.partials, out, nslots, rows, slot_of, out_of, lane);
-  // every arrival is in: re-arm the counter for the next launch (no reply needed)
-  if (lane == 0) asm volatile("st.relaxed.gpu.global.s32 [%0], 0;" ::"l"(prm.counters + wa) : "memory");
 }
 
 // Query row `g` (MMA column) of a segment, or null past the unit's rows.
@@ -799,11 +312,19 @@ struct MmaPath {
         o[mt][3] *= c1;
       }
     }
-    // ---- P^T as the B operand of O^T += V^T P^T
+    // ---- P^T as the B operand of O^T += V^T P^T.  f16 keeps 11 significant
+    // bits of P; bf16 keeps 8, so with bf16 V the weights go in as two parts,
+    // P = hi + lo (each bf16), and the product is taken twice: P's rounding
+    // error drops from 2^-9 to 2^-17 relative, below the fp32 accumulation.
     const uint32_t x0 = kF16 ? dev::pack_f16(p0, p1) : dev::pack_bf16(p0, p1);
     const uint32_t x1 = kF16 ? dev::pack_f16(p2, p3) : dev::pack_bf16(p2, p3);
     const uint32_t pb0 = dev::movm_t(x0);
     const uint32_t pb1 = dev::movm_t(x1);
+    uint32_t pl0 = 0, pl1 = 0;
+    if constexpr (!kF16) {
+      pl0 = dev::movm_t(dev::pack_bf16(p0 - dev::bf16lo_to_f32(x0), p1 - dev::bf16hi_to_f32(x0)));
+      pl1 = dev::movm_t(dev::pack_bf16(p2 - dev::bf16lo_to_f32(x1), p3 - dev::bf16hi_to_f32(x1)));
+    }
     if constexpr (KV == kFP8) {
       const int tok = r8 + ((j & 1) << 3);
       const int add = j >> 1;
@@ -829,6 +350,7 @@ struct MmaPath {
         uint32_t a[4];
         dev::ldsm_x4_t(vs_addr + (mt >> 2) * 2048 + tok * 128 + (((chunk & 7) ^ r8) << 4), a);
         mma(o[mt], a, pb0, pb1);
+        if constexpr (!kF16) mma(o[mt], a, pl0, pl1);
       }
     }
   }
@@ -1102,21 +624,20 @@ using PathFor = typename std::conditional<(G >= 4), MmaPath<KV, ACT, G>, FmaPath
 // Fused append: the K/V rows of `item`'s last token (position len-1) for KV
 // head h.  Lane l < 16 carries elements 8l .. 8l+7 of the K row, lane 16 + l
 // those of the V row (act dtype, 16 bytes).
-// Write those rows into the cache slot of physical block `phys` and into row
+// Write those rows into their cache slot (tile_row + (len-1) % 16) and into row
 // (len-1) % 16 of the staged K and V tiles (the copy brought the block in
 // before the row was written).  Same values as the append kernel: 16-bit rows
 // are copied; FP8 codes are E4M3(rn, satfinite)(fp32(x) * inv_scale).
 template <int KV, int ACT, class Prm>
-__device__ __forceinline__ void append_last_token(const Prm& prm, int h, int len, int32_t phys,
+__device__ __forceinline__ void append_last_token(const Prm& prm, int h, int len, int32_t tile_row,
                                                   uint8_t* st, uint4 val, int lane) {
   using T = Tile<KV>;
   const int r = (len - 1) % kBlock;
   const int kv = lane >> 4, c = lane & 15;
   uint8_t* tile = st + kv * T::kBytes;
   uint8_t* cache = kv ? prm.v_cache : prm.k_cache;
-  const int64_t dst_el =
-      ((static_cast<int64_t>(prm.layer) * prm.num_blocks + phys) * prm.num_kv_heads + h) * kBlock * kHeadDim +
-      static_cast<int64_t>(r) * kHeadDim;
+  // tile_row = cache row of the staged tile's first token slot
+  const int64_t dst_el = (static_cast<int64_t>(tile_row) + r) * kHeadDim;
   if constexpr (KV == kFP8) {
     const float inv = (kv ? prm.v_inv : prm.k_inv)[prm.layer * prm.num_kv_heads + h];
     const uint32_t w[4] = {val.x, val.y, val.z, val.w};
@@ -1356,39 +877,6 @@ cudaError_t dispatch_group(const DecodeKParams<SibPlan>& prm, const CUtensorMap*
 }
 
 template <class PlanT>
-void fill_params(DecodeKParams<PlanT>& prm, const PoolView& pool, const PlanT& plan,
-                 const DecodeArgs& args) {
-  prm.q = static_cast<const uint8_t*>(args.q);
-  prm.out = static_cast<uint8_t*>(args.out);
-  prm.tables = pool.tables;
-  prm.partials = pool.partials;
-  prm.counters = pool.counters;
-  prm.err = pool.err;
-  prm.k_scale = pool.k_scale;
-  prm.v_scale = pool.v_scale;
-  prm.q_item_stride = args.q_item_stride;
-  prm.scale = args.scale;
-  prm.layer = args.layer;
-  prm.num_kv_heads = pool.num_kv_heads;
-  prm.num_blocks = pool.num_blocks;
-  prm.mbps = pool.mbps;
-  prm.group = args.group;
-  prm.total = plan.per_head * pool.num_kv_heads;
-  std::memcpy(&prm.plan, &plan, sizeof(PlanT));
-  // q / out of this launch start at item_offset
-  prm.q += static_cast<int64_t>(args.item_offset) * args.q_item_stride * 2;
-  prm.out += static_cast<int64_t>(args.item_offset) * args.q_item_stride * 2;
-  // fused append: new rows [n][H][128] act dtype, from item_offset on
-  const int64_t kv_off = static_cast<int64_t>(args.item_offset) * pool.num_kv_heads * kHeadDim * 2;
-  prm.k_new = args.k_new ? static_cast<const uint8_t*>(args.k_new) + kv_off : nullptr;
-  prm.v_new = args.v_new ? static_cast<const uint8_t*>(args.v_new) + kv_off : nullptr;
-  prm.k_cache = static_cast<uint8_t*>(pool.k_cache);
-  prm.v_cache = static_cast<uint8_t*>(pool.v_cache);
-  prm.k_inv = pool.k_inv;
-  prm.v_inv = pool.v_inv;
-}
-
-template <class PlanT>
 cudaError_t dispatch_dtypes(const PoolView& pool, const DecodeKParams<PlanT>& prm,
                             const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t stream) {
   if (pool.kv_dtype == kFP8) {
@@ -1414,8 +902,9 @@ cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CU
                           const DecodePlan& plan, const DecodeArgs& args, cudaStream_t stream,
                           int* launches) {
   static thread_local DecodeKParams<DecodePlan> prm;
-  fill_params(prm, pool, plan, args);
-  cudaError_t e = dispatch_dtypes(pool, prm, tmk, tmv, stream);
+  fill_decode_params(prm, pool, plan, args);
+  cudaError_t e = args.use_tc ? launch_decode_tc(pool, tmk, tmv, plan, args, stream)
+                              : dispatch_dtypes(pool, prm, tmk, tmv, stream);
   if (e != cudaSuccess) return e;
   ++*launches;
 
@@ -1441,7 +930,7 @@ cudaError_t launch_decode_sib(const PoolView& pool, const CUtensorMap* tmk, cons
                               const SibPlan& plan, const DecodeArgs& args, cudaStream_t stream,
                               int* launches) {
   static thread_local DecodeKParams<SibPlan> prm;
-  fill_params(prm, pool, plan, args);
+  fill_decode_params(prm, pool, plan, args);
   const cudaError_t e = dispatch_dtypes(pool, prm, tmk, tmv, stream);
   if (e == cudaSuccess) ++*launches;
   return e;

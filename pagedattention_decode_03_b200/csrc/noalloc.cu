@@ -14,12 +14,15 @@
 // scratch -- partial results, arrival counters and an error word -- lives in
 // one file-scope __device__ array of
 // kScratchBytes (12 MiB) that every GPU loading this library holds until the
-// process exits.
+// process exits.  The kernel's bounds checks set bits in the error word (a
+// table entry outside the pool, a bounded wait that gave up); the bits stay
+// set across calls until pa_noalloc_check_errors reads and clears them.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -204,9 +207,10 @@ extern "C" pa_status pa_decode_attention_noalloc(const pa_pool_desc* d, int32_t 
   v.kv_dtype = d->kv_dtype;
   v.act_dtype = d->act_dtype;
 
-  // The scratch keeps the previous call's contents: the arrival counters and
-  // the error word must start at zero.
-  cudaError_t e = cudaMemsetAsync(scratch + kCountersOff, 0, kPartialsOff - kCountersOff, s);
+  // The scratch keeps the previous call's contents: the arrival counters must
+  // start at zero.  The error word is left alone: its bits accumulate until
+  // pa_noalloc_check_errors reads them.
+  cudaError_t e = cudaMemsetAsync(scratch + kCountersOff, 0, sizeof(int32_t) * pa::kMaxWorkers, s);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("cudaMemsetAsync: ") + cudaGetErrorString(e));
 
   const int64_t total = work * d->num_kv_heads;
@@ -233,5 +237,43 @@ extern "C" pa_status pa_decode_attention_noalloc(const pa_pool_desc* d, int32_t 
   int launches = 0;
   e = pa::launch_decode(v, &tmk, &tmv, plan, args, s, &launches);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));
+  return PA_OK;
+}
+
+extern "C" pa_status pa_noalloc_check_errors(int32_t device, void* stream, uint32_t* bits) {
+  pa::set_last_error("");
+  if (!bits) return fail(PA_ERR_INVALID_ARG, "null argument");
+  if (device < 0 || device >= kMaxDevices) return fail(PA_ERR_INVALID_ARG, "device ordinal out of range");
+  {
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    if (!g_scratch_dev[device]) {  // no call on this device yet: nothing to report
+      *bits = 0;
+      return PA_OK;
+    }
+  }
+  int prev = -1;
+  if (cudaGetDevice(&prev) != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice failed");
+  if (prev != device && cudaSetDevice(device) != cudaSuccess) return fail(PA_ERR_CUDA, "cudaSetDevice failed");
+  struct Restore {
+    int prev, dev;
+    ~Restore() {
+      if (prev != dev) cudaSetDevice(prev);
+    }
+  } restore{prev, device};
+  uint8_t* scratch = nullptr;
+  int sms = 0;
+  pa_status st = setup_device(device, &scratch, &sms);
+  if (st != PA_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("cudaStreamSynchronize: ") + cudaGetErrorString(e));
+  uint32_t v = 0;
+  e = cudaMemcpy(&v, scratch + kErrOff, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("read error word: ") + cudaGetErrorString(e));
+  e = cudaMemset(scratch + kErrOff, 0, sizeof(v));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("clear error word: ") + cudaGetErrorString(e));
+  *bits = v;
+  if (v != 0)
+    return fail(PA_ERR_DEVICE_CHECK, "a no-allocation decode call reported device error bits 0x" +
+                                         [v] { char b[16]; std::snprintf(b, sizeof b, "%x", v); return std::string(b); }());
   return PA_OK;
 }

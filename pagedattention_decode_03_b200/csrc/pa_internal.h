@@ -127,6 +127,8 @@ struct DecodeArgs {
   int32_t item_offset;    // index of plan item 0 within the caller's arrays
   const void* k_new;      // fused append: [n][H_kv][128] rows of each item's last token,
   const void* v_new;      // or null (no append)
+  int32_t use_tc = 0;     // plain plans with G = 8 over 16-bit KV: the tcgen05 kernel
+  int32_t l2_ahead = 0;   // tiles prefetched into L2 beyond a worker's staged ones
 };
 
 // Stream-K cost positions per work unit, in KV blocks: they stand for the
@@ -148,6 +150,13 @@ cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CU
 cudaError_t launch_decode_sib(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
                               const SibPlan& plan, const DecodeArgs& args, cudaStream_t stream,
                               int* launches);
+
+// The tcgen05 decode (kernels_decode_tc.cu): plain plans, G = 8, 16-bit KV;
+// one worker per SM.  launch_decode calls it when args.use_tc is set.
+bool decode_tc_applies(int kv_dtype, int group);
+int decode_tc_worker_capacity(int num_sms);
+cudaError_t launch_decode_tc(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                             const DecodePlan& plan, const DecodeArgs& args, cudaStream_t stream);
 
 // Thread-local text returned by pa_last_error() (defined in api.cpp).
 void set_last_error(const std::string& msg);

@@ -1,7 +1,7 @@
 """GPU parity tests: the CUDA path (through the C ABI) against the oracle.
 
 Metadata and cache contents bit-exact; attention within the stated
-tolerance (1e-2 absolute for 16-bit KV, 5e-2 for FP8 KV).  Marked `gpu`.
+tolerance (1e-2 absolute + 1e-2 relative for 16-bit KV, 5e-2 absolute for FP8 KV).  Marked `gpu`.
 """
 import numpy as np
 import pytest
@@ -9,7 +9,7 @@ import torch
 
 import pagedattention_decode_03_b200 as pa
 from oracle import PagedKVOracle, Status, fp8
-from paged_harness import Pair, TOL, from_dev, to_dev
+from paged_harness import Pair, assert_close, from_dev, to_dev
 from workloads import normal_bits, workload
 
 pytestmark = pytest.mark.gpu
@@ -79,10 +79,8 @@ def test_groups_and_ragged_lengths(G, kv):
         for part in (0, -1, 16, 32):
             out = torch.empty_like(q)
             pa.pa_decode_attention(pool, layer, seqs, q, out, 0.0883883461356163, part)
-            got = from_dev(out)
             from oracle.numerics import bits_to_f64
-            err = np.abs(bits_to_f64(got, kv) - ref).max()
-            assert err <= 1e-2, (layer, part, err)
+            assert_close(bits_to_f64(from_dev(out), kv), ref, kv, f"layer {layer}, partition {part}")
     assert pa.pa_check_device_errors(pool) == 0
 
 
@@ -127,7 +125,7 @@ def test_identical_keys_and_constant_values():
     from oracle.numerics import bits_to_f64
     mean_v = bits_to_f64(v, "bf16")[:, 0].mean(axis=0)
     got = bits_to_f64(from_dev(out), "bf16")
-    assert np.abs(got[0] - mean_v).max() <= 1e-2
+    assert_close(got[0], mean_v, "bf16", "identical keys")
     assert np.array_equal(from_dev(out)[1], np.full((H * G, 128), 0x3FC0, np.uint16))
 
 
