@@ -10,7 +10,6 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
-#include <cstdlib>
 #include <optional>
 #include <cstring>
 #include <memory>
@@ -81,10 +80,6 @@ struct DeviceGuard {
   }
 };
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 }  // namespace
 
@@ -100,7 +95,7 @@ struct pa_pool {
   bool host_only = false;
   bool dev_ready = false;
   int num_sms = 0;
-  CUtensorMap tmk{}, tmv{};
+  pa::CacheMaps maps{};
   uint64_t launches = 0;
   // scratch reused across calls
   std::vector<pa::CowPair> cows;
@@ -137,29 +132,10 @@ pa_status ensure_device(pa_pool* p, cudaStream_t stream) {
   e = cudaMemsetAsync(p->view.counters, 0, counter_bytes(p->d), stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(counters)");
 
-  void* fn = nullptr;
-  cudaDriverEntryPointQueryResult q;
-  e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr)
-    return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
-  auto encode = reinterpret_cast<EncodeTiledFn>(fn);
-  const bool fp8 = p->d.kv_dtype == PA_FP8_E4M3;
-  const cuuint64_t rows = static_cast<cuuint64_t>(p->d.num_layers) * p->d.num_blocks *
-                          p->d.num_kv_heads * p->d.block_size;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pa::kHeadDim), rows};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pa::kHeadDim) * (fp8 ? 1 : 2)};
-  // 128-byte rows of the box: 64 x 16-bit or 128 x 8-bit elements, 16 token rows
-  const cuuint32_t box[2] = {fp8 ? 128u : 64u, 16u};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
-  CUresult r = encode(&p->tmk, dt, 2, p->d.k_cache, dims, strides, box, estr,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled(k_cache) failed");
-  r = encode(&p->tmv, dt, 2, p->d.v_cache, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled(v_cache) failed");
+  const int64_t rows = static_cast<int64_t>(p->d.num_layers) * p->d.num_blocks * p->d.num_kv_heads *
+                       p->d.block_size;
+  if (const char* why = pa::encode_cache_maps(p->d.k_cache, p->d.v_cache, p->d.kv_dtype, rows, &p->maps))
+    return fail(PA_ERR_CUDA, why);
   p->dev_ready = true;
   return PA_OK;
 }
@@ -773,11 +749,6 @@ pa_status decode_call(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
   p->last_tc = false;
   pa::DecodeArgs args;
   args.use_tc = 0;
-  static const int l2_ahead = [] {
-    const char* e = std::getenv("PA_L2_AHEAD");
-    return e ? std::atoi(e) : 0;
-  }();
-  args.l2_ahead = l2_ahead;
   args.k_new = k_new;
   args.v_new = v_new;
   args.q = q;
@@ -839,14 +810,14 @@ pa_status decode_call(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
         if (e != cudaSuccess) return cuda_fail(e, "append launch");
         args.k_new = args.v_new = nullptr;
       }
-      e = pa::launch_decode_sib(p->view, &p->tmk, &p->tmv, sib, args, s, &launches);
+      e = pa::launch_decode_sib(p->view, p->maps, sib, args, s, &launches);
       args.k_new = k_new;
       args.v_new = v_new;
       p->last_sets += sib.sets;
       p->last_tiles += (sib.per_head - static_cast<int64_t>(sib.alpha) * sib.nu) * H;
     } else {
       args.use_tc = tc ? 1 : 0;
-      e = pa::launch_decode(p->view, &p->tmk, &p->tmv, plan, args, s, &launches);
+      e = pa::launch_decode(p->view, p->maps, plan, args, s, &launches);
       args.use_tc = 0;
       p->last_tiles += blocks * H;
       p->last_tc = p->last_tc || tc;

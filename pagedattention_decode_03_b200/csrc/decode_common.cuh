@@ -24,7 +24,6 @@ struct DecodeKParams {
   float scale;
   int32_t layer, num_kv_heads, num_blocks, mbps, group;
   int32_t bshift;          // log2(block_size / 16): 0 for 16-token blocks, 1 for 32
-  int32_t l2_ahead;        // tiles a worker prefetches into L2 beyond its staged ones (0: none)
   int64_t total;           // work units over all heads
   // Fused append (null k_new: none): the K/V rows of each item's last token,
   // [n][H][128] act dtype, written into the cache by the worker that reads the
@@ -544,7 +543,6 @@ void fill_decode_params(DecodeKParams<PlanT>& prm, const PoolView& pool, const P
   prm.num_blocks = pool.num_blocks;
   prm.mbps = pool.mbps;
   prm.bshift = pool.block_size == 32 ? 1 : 0;
-  prm.l2_ahead = args.l2_ahead;
   prm.group = args.group;
   prm.total = plan.per_head * pool.num_kv_heads;
   std::memcpy(&prm.plan, &plan, sizeof(PlanT));

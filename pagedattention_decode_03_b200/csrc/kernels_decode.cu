@@ -130,29 +130,9 @@ struct Producer {
       if constexpr (KV == kFP8) {
         dev::tma_load_2d(dst, tmk, 0, row, bar);
         dev::tma_load_2d(dst + Tile<KV>::kBytes, tmv, 0, row, bar);
-      } else {
-        dev::tma_load_2d(dst, tmk, 0, row, bar);
-        dev::tma_load_2d(dst + 2048, tmk, 64, row, bar);
-        dev::tma_load_2d(dst + Tile<KV>::kBytes, tmv, 0, row, bar);
-        dev::tma_load_2d(dst + Tile<KV>::kBytes + 2048, tmv, 64, row, bar);
-      }
-    }
-    // The tile l2_ahead positions further on goes to L2 now, so more of the
-    // worker's reads are in flight than its shared-memory ring holds.
-    const int32_t pb = b + prm.l2_ahead;
-    if (prm.l2_ahead > 0 && pb < seg.b1 && pb - tc_base < 32) {
-      const int32_t pv = __shfl_sync(0xffffffffu, tc_val, pb - tc_base);
-      const int32_t pphys = static_cast<int32_t>(static_cast<uint32_t>(pv) >> 1);
-      if (lane == 0 && static_cast<uint32_t>(pphys) < static_cast<uint32_t>(prm.num_blocks)) {
-        const int32_t prow =
-            (((prm.layer * prm.num_blocks + pphys) * prm.num_kv_heads + seg.h) << (4 + prm.bshift)) +
-            (pv & 1) * kBlock;
-        dev::tma_prefetch_l2_2d(tmk, 0, prow);
-        dev::tma_prefetch_l2_2d(tmv, 0, prow);
-        if constexpr (KV != kFP8) {
-          dev::tma_prefetch_l2_2d(tmk, 64, prow);
-          dev::tma_prefetch_l2_2d(tmv, 64, prow);
-        }
+      } else {  // 3-D boxes: both d-halves of the 16 rows in one copy
+        dev::tma_load_3d(dst, tmk, 0, row, 0, bar);
+        dev::tma_load_3d(dst + Tile<KV>::kBytes, tmv, 0, row, 0, bar);
       }
     }
     ++issued;
@@ -898,13 +878,13 @@ int decode_worker_capacity(int kv_dtype, int /*group*/, int num_sms) {
   return std::min(kMaxWorkers, num_sms * ctas * kWarps);
 }
 
-cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                          const DecodePlan& plan, const DecodeArgs& args, cudaStream_t stream,
-                          int* launches) {
+cudaError_t launch_decode(const PoolView& pool, const CacheMaps& maps, const DecodePlan& plan,
+                          const DecodeArgs& args, cudaStream_t stream, int* launches) {
   static thread_local DecodeKParams<DecodePlan> prm;
   fill_decode_params(prm, pool, plan, args);
-  cudaError_t e = args.use_tc ? launch_decode_tc(pool, tmk, tmv, plan, args, stream)
-                              : dispatch_dtypes(pool, prm, tmk, tmv, stream);
+  // 16-bit tiles come in whole (3-D boxes), FP8 tiles are one 2-D box each
+  cudaError_t e = args.use_tc ? launch_decode_tc(pool, maps, plan, args, stream)
+                              : dispatch_dtypes(pool, prm, &maps.k3, &maps.v3, stream);
   if (e != cudaSuccess) return e;
   ++*launches;
 
@@ -926,12 +906,11 @@ cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CU
   return e;
 }
 
-cudaError_t launch_decode_sib(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                              const SibPlan& plan, const DecodeArgs& args, cudaStream_t stream,
-                              int* launches) {
+cudaError_t launch_decode_sib(const PoolView& pool, const CacheMaps& maps, const SibPlan& plan,
+                              const DecodeArgs& args, cudaStream_t stream, int* launches) {
   static thread_local DecodeKParams<SibPlan> prm;
   fill_decode_params(prm, pool, plan, args);
-  const cudaError_t e = dispatch_dtypes(pool, prm, tmk, tmv, stream);
+  const cudaError_t e = dispatch_dtypes(pool, prm, &maps.k3, &maps.v3, stream);
   if (e == cudaSuccess) ++*launches;
   return e;
 }

@@ -58,16 +58,21 @@ constexpr int kTcStage = 2 * kTcKV;            // K and V (64 KB)
 constexpr int kTcQ = 4096;                     // [2 d-halves][16 rows][128 B]
 constexpr int kTcP = 4096;                     // P^T: [16 token groups][2 column blocks][8][8]
 constexpr int kTcCols = 64;                    // TMEM: S^T x 2 buffers (16 each), O^T (16)
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 224;
 constexpr int kTcSoftmax = 128;                // threads of warps 2..5
 
 // shared-memory map (offsets from a 1024-byte aligned base)
 constexpr int kOffQ = kTcStages * kTcStage;                  // 2 Q buffers
-constexpr int kOffP = kOffQ + 2 * kTcQ;
-constexpr int kOffBar = kOffP + kTcP;
-// barriers: full[3] empty[3] qfull[2] qempty[2] sfull[2] sempty[2] pfull obar done
+constexpr int kOffP = kOffQ + 2 * kTcQ;                      // 2 P buffers (by tile parity)
+constexpr int kOffBar = kOffP + 2 * kTcP;
+// barriers: full[3] empty[3] qfull[2] qempty[2] sfull[2] sempty[2] pfull[2] obar[2] done
+// part[2]; pfull[b] / obar[b] complete with the softmax / P.V of each tile of
+// parity b (the softmax may run one tile ahead of the MMA warp's wait, so one
+// barrier would let two phases complete under one parity); part[k] completes
+// once, when the partial result of slot 2w + k is written
 constexpr int kBarFull = 0, kBarEmpty = 3, kBarQFull = 6, kBarQEmpty = 8, kBarSFull = 10,
-              kBarSEmpty = 12, kBarPFull = 14, kBarO = 15, kBarDone = 16, kNumBars = 17;
+              kBarSEmpty = 12, kBarPFull = 14, kBarO = 16, kBarDone = 18, kBarPart = 19,
+              kNumBars = 21;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;              // TMEM base address
 constexpr int kOffRows = kOffTmem + 8;                        // cache row of each staged tile [3][8]
 constexpr int kOffRed = kOffRows + kTcStages * kTcTiles * 4;  // reductions [2][4][8] x 2
@@ -213,8 +218,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       dev::mbar_init(bar(kBarSEmpty + b), 4);
     }
     dev::mbar_init(bar(kBarPFull), 4);
+    dev::mbar_init(bar(kBarPFull + 1), 4);
     dev::mbar_init(bar(kBarO), 1);
+    dev::mbar_init(bar(kBarO + 1), 1);
     dev::mbar_init(bar(kBarDone), 1);
+    dev::mbar_init(bar(kBarPart), 4);
+    dev::mbar_init(bar(kBarPart + 1), 4);
     dev::fence_mbar_init();
     dev::tma_prefetch_desc(&tmk);
     dev::tma_prefetch_desc(&tmv);
@@ -272,49 +281,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         if (lane == 0) dev::mbar_arrive_expect_tx(bar(kBarFull + st), t.n * 8192);
-        for (int j = 0; j < t.n; ++j) {
-          const int32_t bj = b + j;
-          if (s.k != tc_unit || bj < tc_base || bj >= tc_base + 32) {
-            tc_unit = s.k;
-            tc_base = bj;
-            const BlockRef r = locate<8>(prm, s, bj + lane);
-            const int32_t e = r.b >> prm.bshift;
-            int32_t v = r.b >= 0 && e < prm.mbps ? prm.tables[static_cast<int64_t>(r.seq) * prm.mbps + e] : 0;
-            tc_val = static_cast<int32_t>((static_cast<uint32_t>(v) << 1) |
-                                          static_cast<uint32_t>(r.b & ((1 << prm.bshift) - 1)));
-          }
-          const int32_t tv = __shfl_sync(0xffffffffu, tc_val, bj - tc_base);
+        __syncwarp();  // the expected bytes are counted before any copy is issued
+        // physical ids of blocks b .. b + n - 1 (the lane cache holds 32 of the unit's)
+        if (s.k != tc_unit || b < tc_base || b + t.n > tc_base + 32) {
+          tc_unit = s.k;
+          tc_base = b;
+          const BlockRef r = locate<8>(prm, s, b + lane);
+          const int32_t e = r.b >> prm.bshift;
+          int32_t v = r.b >= 0 && e < prm.mbps ? prm.tables[static_cast<int64_t>(r.seq) * prm.mbps + e] : 0;
+          tc_val = static_cast<int32_t>((static_cast<uint32_t>(v) << 1) |
+                                        static_cast<uint32_t>(r.b & ((1 << prm.bshift) - 1)));
+        }
+        // lane j issues block j's four copies: the copies of a tile go out in
+        // parallel rather than one after another from a single lane
+        const int32_t tv = __shfl_sync(0xffffffffu, tc_val, (b - tc_base + lane) & 31);
+        if (lane < t.n) {
           int32_t phys = static_cast<int32_t>(static_cast<uint32_t>(tv) >> 1);
           if (static_cast<uint32_t>(phys) >= static_cast<uint32_t>(prm.num_blocks)) {
-            if (lane == 0) atomicOr(prm.err, kErrBadBlock);
+            atomicOr(prm.err, kErrBadBlock);
             phys = 0;
           }
           const int32_t row =
               (((prm.layer * prm.num_blocks + phys) * prm.num_kv_heads + s.h) << (4 + prm.bshift)) +
               (tv & 1) * kBlock;
-          if (lane == 0) {
-            rows_s[st * kTcTiles + j] = row;
-            const uint32_t dst = base + st * kTcStage + j * 2048;
-            dev::tma_load_2d(dst, &tmk, 0, row, bar(kBarFull + st));
-            dev::tma_load_2d(dst + kTcHalf, &tmk, 64, row, bar(kBarFull + st));
-            dev::tma_load_2d(dst + kTcKV, &tmv, 0, row, bar(kBarFull + st));
-            dev::tma_load_2d(dst + kTcKV + kTcHalf, &tmv, 64, row, bar(kBarFull + st));
-          }
-        }
-        // the blocks after this tile go to L2 now (more reads in flight than
-        // the shared-memory ring holds)
-        for (int32_t pb = b + t.n; pb < min(s.b1, b + t.n + prm.l2_ahead) && pb - tc_base < 32; ++pb) {
-          const int32_t pv = __shfl_sync(0xffffffffu, tc_val, pb - tc_base);
-          const int32_t pphys = static_cast<int32_t>(static_cast<uint32_t>(pv) >> 1);
-          if (lane == 0 && static_cast<uint32_t>(pphys) < static_cast<uint32_t>(prm.num_blocks)) {
-            const int32_t prow =
-                (((prm.layer * prm.num_blocks + pphys) * prm.num_kv_heads + s.h) << (4 + prm.bshift)) +
-                (pv & 1) * kBlock;
-            dev::tma_prefetch_l2_2d(&tmk, 0, prow);
-            dev::tma_prefetch_l2_2d(&tmk, 64, prow);
-            dev::tma_prefetch_l2_2d(&tmv, 0, prow);
-            dev::tma_prefetch_l2_2d(&tmv, 64, prow);
-          }
+          rows_s[st * kTcTiles + lane] = row;
+          const uint32_t dst = base + st * kTcStage + lane * 2048;
+          dev::tma_load_2d(dst, &tmk, 0, row, bar(kBarFull + st));
+          dev::tma_load_2d(dst + kTcHalf, &tmk, 64, row, bar(kBarFull + st));
+          dev::tma_load_2d(dst + kTcKV, &tmv, 0, row, bar(kBarFull + st));
+          dev::tma_load_2d(dst + kTcKV + kTcHalf, &tmv, 64, row, bar(kBarFull + st));
         }
         ++tile_i;
       }
@@ -332,102 +327,133 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr bool kBf = ACT == kBF16;
     constexpr uint32_t kIdS = instr_desc(kBf, false, false, 128, 16);
     constexpr uint32_t kIdO = instr_desc(kBf, true, true, 128, 16);
-    uint32_t tile_i = 0, seg_i = 0;
-    // the previous tile, whose P.V waits for the softmax of that tile
-    bool have_prev = false, prev_first = false;
-    uint32_t prev_st = 0, prev_i = 0;
-    int32_t prev_n = 0;
-    auto issue_pv = [&]() -> bool {
-      if (!warp_wait(bar(kBarPFull), prev_i & 1)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t vbase = base + prev_st * kTcStage + kTcKV;
-        const uint32_t pbase = base + kOffP;
-        for (int j = 0; j < prev_n; ++j)
-          umma(tmem + 32, smem_desc(vbase + j * 2048, kPvALbo, kPvASbo, kLayoutSW128),
-               smem_desc(pbase + j * 512, kPvBLbo, kPvBSbo, kLayoutNone), kIdO, !(prev_first && j == 0));
-        umma_commit(bar(kBarO));
-        umma_commit(bar(kBarEmpty + prev_st));
-      }
-      __syncwarp();
-      return true;
+    // An event loop: the P.V of the oldest tile whose softmax is done, and the
+    // S of the next tile whose data, S buffer and query rows are in, each
+    // issued as soon as it can go (a P.V never waits for a later tile's copy,
+    // so a stage is released as early as possible).
+    struct PvTile {
+      uint32_t st;
+      int32_t n;
+      bool first;
     };
-    for (;;) {
-      const Seg s = cur.next(prm);
-      if (!s.valid) break;
-      const uint32_t qb = seg_i & 1;
-      if (!warp_wait(bar(kBarQFull + qb), (seg_i >> 1) & 1)) {
+    PvTile ring[4];
+    uint32_t ns = 0, np = 0, seg_i = 0;   // tiles whose S / P.V went out; segments started
+    bool s_done = false, q_ready = false;
+    Seg s;
+    int32_t b = 0;
+    auto next_segment = [&]() {
+      s = cur.next(prm);
+      s_done = !s.valid;
+      b = s.b0;
+      q_ready = false;
+    };
+    auto ready = [&](int idx, uint32_t parity) {
+      return __any_sync(0xffffffffu, dev::mbar_test_wait(bar(idx), parity));
+    };
+    next_segment();
+    uint32_t idle = 0;
+    while (!s_done || np < ns) {
+      bool progress = false;
+      if (np < ns && ready(kBarPFull + (np & 1), (np >> 1) & 1)) {
+        tc_fence_after();
+        const PvTile& pt = ring[np & 3];
+        if (lane == 0) {
+          const uint32_t vbase = base + pt.st * kTcStage + kTcKV;
+          const uint32_t pbase = base + kOffP + (np & 1) * kTcP;
+          for (int j = 0; j < pt.n; ++j)
+            umma(tmem + 32, smem_desc(vbase + j * 2048, kPvALbo, kPvASbo, kLayoutSW128),
+                 smem_desc(pbase + j * 512, kPvBLbo, kPvBSbo, kLayoutNone), kIdO, !(pt.first && j == 0));
+          umma_commit(bar(kBarO + (np & 1)));
+          umma_commit(bar(kBarEmpty + pt.st));
+        }
+        __syncwarp();
+        ++np;
+        progress = true;
+      }
+      if (!s_done && ns - np < 3) {
+        const uint32_t qb = seg_i & 1;
+        const uint32_t st = ns % kTcStages;
+        if (!q_ready) q_ready = ready(kBarQFull + qb, (seg_i >> 1) & 1);
+        if (q_ready && ready(kBarFull + st, (ns / kTcStages) & 1) &&
+            ready(kBarSEmpty + (ns & 1), ((ns >> 1) & 1) ^ 1)) {
+          const TcTile t = tile_of(s, b);
+          const uint32_t kst = base + st * kTcStage;
+          uint8_t* kst_p = sm + st * kTcStage;
+          // the item's last block in this tile: fused append row, V rows past the length
+          const int32_t last = (s.len - 1) / kBlock - b;
+          if (last >= 0 && last < t.n) {
+            const int r = (s.len - 1) % kBlock;
+            if (prm.k_new != nullptr) {
+              const int kv = lane >> 4, c = lane & 15;
+              const uint4 val = __ldcg(new_row_ptr(prm, s.h, s.i, lane));
+              uint8_t* tile = kst_p + kv * kTcKV + (c >> 3) * kTcHalf + last * 2048;
+              *reinterpret_cast<uint4*>(tile + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = val;
+              uint8_t* cache = kv ? prm.v_cache : prm.k_cache;
+              const int64_t dst_el =
+                  (static_cast<int64_t>(rows_s[st * kTcTiles + last]) + r) * kHeadDim + c * 8;
+              *reinterpret_cast<uint4*>(cache + dst_el * 2) = val;
+            }
+            const int nvalid = r + 1;
+            for (int c = lane; c < (kBlock - nvalid) * 16; c += 32) {
+              const int tr = nvalid + c / 16, k = c % 16;
+              *reinterpret_cast<uint4*>(kst_p + kTcKV + (k >> 3) * kTcHalf + last * 2048 + tr * 128 +
+                                        ((k & 7) << 4)) = make_uint4(0, 0, 0, 0);
+            }
+            dev::fence_proxy_async_smem();
+          }
+          __syncwarp();
+          tc_fence_after();
+          const uint32_t sb = ns & 1;
+          const bool seg_last = b + kTcTiles >= s.b1;
+          if (lane == 0) {
+            const uint32_t qbase = base + kOffQ + qb * kTcQ;
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t ka = kst + (kk >> 2) * kTcHalf + (kk & 3) * 32;
+              const uint32_t qa = qbase + (kk >> 2) * 2048 + (kk & 3) * 32;
+              umma(tmem + sb * 16, smem_desc(ka, 16, 1024, kLayoutSW128),
+                   smem_desc(qa, 16, 1024, kLayoutSW128), kIdS, kk > 0);
+            }
+            umma_commit(bar(kBarSFull + sb));
+            if (seg_last) umma_commit(bar(kBarQEmpty + qb));  // last S of the segment
+          }
+          __syncwarp();
+          ring[ns & 3] = PvTile{st, t.n, b == s.b0};
+          ++ns;
+          b += kTcTiles;
+          if (seg_last) {
+            ++seg_i;
+            next_segment();
+          }
+          progress = true;
+        }
+      }
+      if (progress) {
+        idle = 0;
+      } else if (++idle > kWaitLimit) {
         failed = true;
         break;
       }
-      for (int32_t b = s.b0; b < s.b1; b += kTcTiles) {
-        const TcTile t = tile_of(s, b);
-        const uint32_t st = tile_i % kTcStages;
-        if (!warp_wait(bar(kBarFull + st), (tile_i / kTcStages) & 1)) {
-          failed = true;
-          break;
-        }
-        const uint32_t kst = base + st * kTcStage;
-        uint8_t* kst_p = sm + st * kTcStage;
-        // the item's last block in this tile: fused append row, V rows past the length
-        const int32_t last = (s.len - 1) / kBlock - b;
-        if (last >= 0 && last < t.n) {
-          const int r = (s.len - 1) % kBlock;
-          if (prm.k_new != nullptr) {
-            const int kv = lane >> 4, c = lane & 15;
-            const uint4 val = __ldcg(new_row_ptr(prm, s.h, s.i, lane));
-            uint8_t* tile = kst_p + kv * kTcKV + (c >> 3) * kTcHalf + last * 2048;
-            *reinterpret_cast<uint4*>(tile + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = val;
-            uint8_t* cache = kv ? prm.v_cache : prm.k_cache;
-            const int64_t dst_el = (static_cast<int64_t>(rows_s[st * kTcTiles + last]) + r) * kHeadDim + c * 8;
-            *reinterpret_cast<uint4*>(cache + dst_el * 2) = val;
-          }
-          const int nvalid = r + 1;
-          for (int c = lane; c < (kBlock - nvalid) * 16; c += 32) {
-            const int tr = nvalid + c / 16, k = c % 16;
-            *reinterpret_cast<uint4*>(kst_p + kTcKV + (k >> 3) * kTcHalf + last * 2048 + tr * 128 +
-                                      ((k & 7) << 4)) = make_uint4(0, 0, 0, 0);
-          }
-          dev::fence_proxy_async_smem();
-        }
-        __syncwarp();
-        const uint32_t sb = tile_i & 1;
-        if (!warp_wait(bar(kBarSEmpty + sb), ((tile_i >> 1) & 1) ^ 1)) {
-          failed = true;
-          break;
-        }
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t qbase = base + kOffQ + qb * kTcQ;
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t ka = kst + (kk >> 2) * kTcHalf + (kk & 3) * 32;
-            const uint32_t qa = qbase + (kk >> 2) * 2048 + (kk & 3) * 32;
-            umma(tmem + sb * 16, smem_desc(ka, 16, 1024, kLayoutSW128), smem_desc(qa, 16, 1024, kLayoutSW128),
-                 kIdS, kk > 0);
-          }
-          umma_commit(bar(kBarSFull + sb));
-          if (b + kTcTiles >= s.b1) umma_commit(bar(kBarQEmpty + qb));  // last S of the segment
-        }
-        __syncwarp();
-        if (have_prev && !issue_pv()) {
-          failed = true;
-          break;
-        }
-        have_prev = true;
-        prev_first = b == s.b0;
-        prev_st = st;
-        prev_i = tile_i;
-        prev_n = t.n;
-        ++tile_i;
-      }
-      if (failed) break;
-      ++seg_i;
     }
-    if (!failed && have_prev && !issue_pv()) failed = true;
     // every MMA issued has finished before the tensor memory is released
     if (lane == 0) umma_commit(bar(kBarDone));
     __syncwarp();
     warp_wait(bar(kBarDone), 0);
+  } else if (warp == 6) {
+    // ================================================================ merge
+    // A worker writes at most one partial to slot 2w (its share starts inside
+    // a unit) and one to slot 2w + 1 (its share ends inside one).
+    if (prm.plan.mode == kSplitStreamK) {
+      for (;;) {
+        const Seg s = cur.next(prm);
+        if (!s.valid) break;
+        if (s.dest < 0) continue;
+        if (!warp_wait(bar(kBarPart + (s.dest & 1)), 0)) {
+          failed = true;
+          break;
+        }
+        settle_partial<ACT, 8, 8>(prm, s, 8, lane);
+      }
+    }
   } else {
     // ======================================================= softmax, epilogue
     const int sw = warp - 2;                    // softmax warp 0..3
@@ -436,7 +462,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float sl2 = prm.scale * kLog2e;
     uint32_t tile_i = 0, seg_i = 0;
-    uint8_t* pbuf = sm + kOffP;
+    // the P.V of tile i completes phase (i >> 1) of obar[i & 1]
+    auto pv_done = [&](uint32_t i) {
+      return dev::mbar_wait_bounded(bar(kBarO + (i & 1)), (i >> 1) & 1, kWaitLimit);
+    };
     // `failed` may differ between the softmax warps until the next barrier ORs
     // it over them; `abort` is that agreed value, the same in every warp
     bool abort = false;
@@ -502,10 +531,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           p[g] = dev::exp2_approx(x[g] - mref[g]);
           lpart[g] = lpart[g] * corr[g] + p[g];
         }
-        // P.V of the previous tile reads the P buffer and accumulates into O
-        if (tile_i > 0) ok = dev::mbar_wait_bounded(bar(kBarO), (tile_i - 1) & 1, kWaitLimit);
+        // O is rescaled between the P.V of the previous tile and this one's;
+        // otherwise only this tile's P buffer must be free (the P.V of two
+        // tiles back), so this softmax overlaps the previous tile's P.V
+        const bool rescale_o = rescale && b != s.b0;
+        if (rescale_o) {
+          ok = pv_done(tile_i - 1);
+        } else if (tile_i > 1) {
+          ok = pv_done(tile_i - 2);
+        }
         tc_fence_after();
-        if (rescale && b != s.b0) {
+        if (rescale_o) {
           float o[16];
           tmem_ld16(tl + 32, o);
 #pragma unroll
@@ -523,19 +559,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             lo[k] = dev::pack_f16(p[2 * k] - dev::f16lo_to_f32(hi[k]), p[2 * k + 1] - dev::f16hi_to_f32(hi[k]));
           }
         }
-        uint8_t* pt = pbuf + (t >> 3) * 256 + (t & 7) * 16;
+        uint8_t* pt = sm + kOffP + (tile_i & 1) * kTcP + (t >> 3) * 256 + (t & 7) * 16;
         *reinterpret_cast<uint4*>(pt) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<uint4*>(pt + 128) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         dev::fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kBarPFull));
+        if (lane == 0) mbar_arrive(bar(kBarPFull + (tile_i & 1)));
         failed |= !ok;   // agreed on at the next barrier
         ++tile_i;
       }
       if (abort) break;
       // ---- epilogue: the segment's last P.V, the row sums, the output
-      bool ok = !failed && dev::mbar_wait_bounded(bar(kBarO), (tile_i - 1) & 1, kWaitLimit);
+      bool ok = !failed && pv_done(tile_i - 1);
       tc_fence_after();
       float oc[16];
       tmem_ld16(tl + 32, oc);
@@ -570,9 +606,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int g = 0; g < 8; ++g)
             *reinterpret_cast<float2*>(slot + kMaxGroup * kHeadDim + 2 * g) = make_float2(mref[g], lt[g]);
         }
-        __threadfence();
-        softmax_bar_or(false);
-        if (sw == 0) settle_partial<ACT, 8, 8>(prm, s, 8, lane);
+        if (prm.plan.mode == kSplitStreamK) {
+          // the merge warp counts this partial in (and merges, if last) while
+          // the softmax goes on with the next segment
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kBarPart + (s.dest & 1)));
+        }
       }
       ++seg_i;
     }
@@ -624,8 +664,8 @@ cudaError_t run_tc(const TcParams& tp, const CUtensorMap* tmk, const CUtensorMap
 
 bool decode_tc_applies(int kv_dtype, int group) { return group == 8 && kv_dtype != kFP8; }
 
-cudaError_t launch_decode_tc(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                             const DecodePlan& plan, const DecodeArgs& args, cudaStream_t stream) {
+cudaError_t launch_decode_tc(const PoolView& pool, const CacheMaps& maps, const DecodePlan& plan,
+                             const DecodeArgs& args, cudaStream_t stream) {
   if (!decode_tc_applies(pool.kv_dtype, args.group)) return cudaErrorInvalidValue;
   EncodeTiledFn encode = tc_encoder();
   if (!encode) return cudaErrorNotSupported;
@@ -643,8 +683,8 @@ cudaError_t launch_decode_tc(const PoolView& pool, const CUtensorMap* tmk, const
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  return pool.act_dtype == kBF16 ? run_tc<kBF16>(tp, tmk, tmv, tmq, stream)
-                                 : run_tc<kFP16>(tp, tmk, tmv, tmq, stream);
+  return pool.act_dtype == kBF16 ? run_tc<kBF16>(tp, &maps.k, &maps.v, tmq, stream)
+                                 : run_tc<kFP16>(tp, &maps.k, &maps.v, tmq, stream);
 }
 
 int decode_tc_worker_capacity(int num_sms) { return std::min(kMaxWorkers, num_sms); }

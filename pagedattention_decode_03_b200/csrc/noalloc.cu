@@ -57,11 +57,6 @@ pa_status fail(pa_status s, const std::string& m) {
   return s;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
 // Once per device, with that device current: the scratch's device address
 // and the SM count.
 pa_status setup_device(int dev, uint8_t** scratch, int* sms) {
@@ -81,19 +76,6 @@ pa_status setup_device(int dev, uint8_t** scratch, int* sms) {
   *scratch = g_scratch_dev[dev];
   *sms = g_num_sms[dev];
   return PA_OK;
-}
-
-EncodeTiledFn encoder() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
 }
 
 }  // namespace
@@ -166,24 +148,10 @@ extern "C" pa_status pa_decode_attention_noalloc(const pa_pool_desc* d, int32_t 
   int sms = 0;
   pa_status st = setup_device(dev, &scratch, &sms);
   if (st != PA_OK) return st;
-  EncodeTiledFn encode = encoder();
-  if (!encode) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
-
-  const bool fp8 = d->kv_dtype == PA_FP8_E4M3;
-  const cuuint64_t rows = static_cast<cuuint64_t>(d->num_layers) * d->num_blocks * d->num_kv_heads * 16;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pa::kHeadDim), rows};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pa::kHeadDim) * (fp8 ? 1 : 2)};
-  const cuuint32_t box[2] = {fp8 ? 128u : 64u, 16u};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
-  CUtensorMap tmk, tmv;
-  if (encode(&tmk, dt, 2, d->k_cache, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
-      encode(&tmv, dt, 2, d->v_cache, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  pa::CacheMaps maps;
+  const int64_t rows = static_cast<int64_t>(d->num_layers) * d->num_blocks * d->num_kv_heads * 16;
+  if (const char* why = pa::encode_cache_maps(d->k_cache, d->v_cache, d->kv_dtype, rows, &maps))
+    return fail(PA_ERR_CUDA, why);
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   pa::PoolView v{};
@@ -235,7 +203,7 @@ extern "C" pa_status pa_decode_attention_noalloc(const pa_pool_desc* d, int32_t 
   args.q_item_stride = static_cast<int64_t>(num_q_heads) * pa::kHeadDim;
   args.item_offset = 0;
   int launches = 0;
-  e = pa::launch_decode(v, &tmk, &tmv, plan, args, s, &launches);
+  e = pa::launch_decode(v, maps, plan, args, s, &launches);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));
   return PA_OK;
 }

@@ -128,7 +128,6 @@ struct DecodeArgs {
   const void* k_new;      // fused append: [n][H_kv][128] rows of each item's last token,
   const void* v_new;      // or null (no append)
   int32_t use_tc = 0;     // plain plans with G = 8 over 16-bit KV: the tcgen05 kernel
-  int32_t l2_ahead = 0;   // tiles prefetched into L2 beyond a worker's staged ones
 };
 
 // Stream-K cost positions per work unit, in KV blocks: they stand for the
@@ -143,20 +142,28 @@ inline int32_t stream_k_alpha(int32_t /*kv_dtype*/) { return 12; }
 int decode_worker_capacity(int kv_dtype, int group, int num_sms);
 int decode_warps_per_cta();
 
-cudaError_t launch_decode(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                          const DecodePlan& plan, const DecodeArgs& args, cudaStream_t stream,
-                          int* launches);
+// TMA tensor maps of a cache (tensor_maps.cpp): the 2-D view [rows][128] with
+// boxes of 16 rows x 128 bytes, and for 16-bit caches the 3-D view
+// [2 d-halves][rows][64] whose box {64, 16, 2} is a whole 16-row tile.
+struct CacheMaps {
+  CUtensorMap k, v;
+  CUtensorMap k3, v3;  // copies of k / v for FP8 caches
+};
+// Returns null on success, else what failed.
+const char* encode_cache_maps(void* k_cache, void* v_cache, int kv_dtype, int64_t rows, CacheMaps* maps);
+
+cudaError_t launch_decode(const PoolView& pool, const CacheMaps& maps, const DecodePlan& plan,
+                          const DecodeArgs& args, cudaStream_t stream, int* launches);
 // Same for a plan with shared entries; group must be 1, 2 or 4.
-cudaError_t launch_decode_sib(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                              const SibPlan& plan, const DecodeArgs& args, cudaStream_t stream,
-                              int* launches);
+cudaError_t launch_decode_sib(const PoolView& pool, const CacheMaps& maps, const SibPlan& plan,
+                              const DecodeArgs& args, cudaStream_t stream, int* launches);
 
 // The tcgen05 decode (kernels_decode_tc.cu): plain plans, G = 8, 16-bit KV;
 // one worker per SM.  launch_decode calls it when args.use_tc is set.
 bool decode_tc_applies(int kv_dtype, int group);
 int decode_tc_worker_capacity(int num_sms);
-cudaError_t launch_decode_tc(const PoolView& pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                             const DecodePlan& plan, const DecodeArgs& args, cudaStream_t stream);
+cudaError_t launch_decode_tc(const PoolView& pool, const CacheMaps& maps, const DecodePlan& plan,
+                             const DecodeArgs& args, cudaStream_t stream);
 
 // Thread-local text returned by pa_last_error() (defined in api.cpp).
 void set_last_error(const std::string& msg);

@@ -41,7 +41,7 @@ def group8(kv="bf16", block=16, lens=LENS, cfg=20):
 
 
 def tc_pair(w, **kw):
-    p = Pair(w, min_partition=16, **kw)
+    p = Pair(w, min_partition=max(16, w.block_size), **kw)
     pa.pa_set_decode_path(p.pool, "tcgen05")
     return p
 
