@@ -374,9 +374,19 @@ def steps_of(a):
 
 def run_ours(a, rank, world, local_rank):
     import torch
-    import workloads
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
+    # All work of the replica runs on a stream of its own, as in a serving
+    # engine: the library then launches each kernel with programmatic stream
+    # serialization, so a decode launch's prologue overlaps the tail of the
+    # previous one (on the legacy default stream every launch waits for the
+    # previous kernel to end).
+    with torch.cuda.stream(torch.cuda.Stream(device)):
+        return _run_ours(a, rank, world, local_rank, device)
+
+
+def _run_ours(a, rank, world, local_rank, device):
+    import torch
     from pagedattention_decode_03_b200 import build as _b
     if rank == 0 or world == 1:
         _b.build()
