@@ -487,12 +487,99 @@ __device__ __forceinline__ int atom_add_acq_rel(int32_t* p, int32_t v) {
   return old;
 }
 
+// Shared memory a merging warp may stage partial slots in: a worker's copy
+// ring once no copy of its own is in flight.  slots = 0: merge from registers.
+struct MergeStage {
+  uint8_t* ptr;
+  uint32_t addr;      // shared-state address of ptr
+  int slots;          // whole partial slots that fit
+  uint32_t bar;       // an mbarrier of this warp for the staging copies
+  uint32_t* phase;    // its phase count
+};
+
+constexpr uint32_t kSlotBytes = sizeof(float) * kPartialSlotFloats;
+
+// merge_unit_warp with the slots brought into shared memory by bulk copies,
+// stage.slots at a time (one copy per slot, all in flight together), so a
+// merge of n slots takes ceil(n / stage.slots) round trips to L2 instead of
+// one per two slots.  Same arithmetic, same slot order, so the same result
+// bit for bit.  False if a copy wait gave up (nothing was written).
+template <int ACT, int R, class SlotFn, class OutFn>
+__device__ __forceinline__ bool merge_unit_warp_staged(const float* partials, uint16_t* out, int nslots,
+                                                       int rows, SlotFn slot_of, OutFn out_of, int lane,
+                                                       const MergeStage& st) {
+  float M[R], L[R];
+  float4 acc[R];
+#pragma unroll
+  for (int gg = 0; gg < R; ++gg) {
+    M[gg] = -INFINITY;
+    L[gg] = 0.f;
+    acc[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // the arrivals' acquire comes before the copies' reads; the ring's last
+  // reads come before the copies' writes
+  dev::fence_proxy_async_global();
+  dev::fence_proxy_async_smem();
+  for (int k0 = 0; k0 < nslots; k0 += st.slots) {
+    const int cnt = min(st.slots, nslots - k0);
+    if (lane == 0) dev::mbar_arrive_expect_tx(st.bar, cnt * kSlotBytes);
+    __syncwarp();
+    if (lane < cnt)
+      dev::bulk_load(st.addr + lane * kSlotBytes,
+                     partials + static_cast<int64_t>(slot_of(k0 + lane)) * kPartialSlotFloats, kSlotBytes, st.bar);
+    const bool ok = dev::mbar_wait_bounded(st.bar, *st.phase & 1u, kWaitLimit);
+    if (!__all_sync(0xffffffffu, ok)) {
+      // let the copies land before the ring can be reused or released
+      dev::mbar_wait_bounded(st.bar, *st.phase & 1u, kWaitLimit);
+      ++*st.phase;
+      return false;
+    }
+    ++*st.phase;
+    for (int j = 0; j < cnt; ++j) {
+      const float* slot = reinterpret_cast<const float*>(st.ptr + j * kSlotBytes);
+#pragma unroll
+      for (int gg = 0; gg < R; ++gg) {
+        if (gg < rows) {
+          const float2 ml = *reinterpret_cast<const float2*>(slot + kMaxGroup * kHeadDim + 2 * gg);
+          const float4 x = *reinterpret_cast<const float4*>(slot + gg * kHeadDim + 4 * lane);
+          const float mn = fmaxf(M[gg], ml.x);
+          const float ref = mn == -INFINITY ? 0.f : mn;
+          const float a = dev::exp2_approx(M[gg] - ref);
+          const float b = dev::exp2_approx(ml.x - ref);
+          M[gg] = mn;
+          L[gg] = L[gg] * a + ml.y * b;
+          acc[gg].x = acc[gg].x * a + x.x * b;
+          acc[gg].y = acc[gg].y * a + x.y * b;
+          acc[gg].z = acc[gg].z * a + x.z * b;
+          acc[gg].w = acc[gg].w * a + x.w * b;
+        }
+      }
+    }
+    __syncwarp();  // every lane is done with the stage before it is refilled
+    dev::fence_proxy_async_smem();
+  }
+#pragma unroll
+  for (int gg = 0; gg < R; ++gg) {
+    if (gg < rows) {
+      const float inv = 1.f / L[gg];
+      const uint32_t a = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].x * inv)) |
+                         (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].y * inv)) << 16);
+      const uint32_t b = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].z * inv)) |
+                         (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].w * inv)) << 16);
+      *reinterpret_cast<uint2*>(out + out_of(gg) + 4 * lane) = make_uint2(a, b);
+    }
+  }
+  return true;
+}
+
 // Stream-K: after a worker wrote the partial of a cut unit, it counts itself
 // in; the last of the unit's workers merges all of them into the output and
 // re-arms the counter.  (Counter = the unit's first worker, unique per cut
-// unit.)  R = row capacity of the merge (rows <= R).
+// unit.)  R = row capacity of the merge (rows <= R).  With stage.slots > 0
+// the merge stages the slots in shared memory (merge_unit_warp_staged).
 template <int ACT, int G, int R, class Prm>
-__device__ __forceinline__ void settle_partial(const Prm& prm, const Seg& s, int rows, int lane) {
+__device__ __forceinline__ void settle_partial(const Prm& prm, const Seg& s, int rows, int lane,
+                                               const MergeStage& stage = MergeStage{nullptr, 0, 0, 0, nullptr}) {
   const auto& P = prm.plan;
   if (plan_mode(P) != kSplitStreamK) return;  // fixed partitions: a separate reduce kernel merges
   const int W = P.workers;
@@ -518,7 +605,13 @@ __device__ __forceinline__ void settle_partial(const Prm& prm, const Seg& s, int
   };
   auto out_of = [&](int r) { return row_offset<G>(prm, s, r); };
   uint16_t* out = reinterpret_cast<uint16_t*>(prm.out);
-  merge_unit_warp<ACT, R>(prm.partials, out, nslots, rows, slot_of, out_of, lane);
+  if (stage.slots > 0) {
+    if (!merge_unit_warp_staged<ACT, R>(prm.partials, out, nslots, rows, slot_of, out_of, lane, stage) &&
+        lane == 0)
+      atomicOr(prm.err, kErrTimeout);
+  } else {
+    merge_unit_warp<ACT, R>(prm.partials, out, nslots, rows, slot_of, out_of, lane);
+  }
   // every arrival is in: re-arm the counter for the next launch (no reply needed)
   if (lane == 0) asm volatile("st.relaxed.gpu.global.s32 [%0], 0;" ::"l"(prm.counters + wa) : "memory");
 }

@@ -342,7 +342,7 @@ struct MmaPath {
   }
 
   template <class Prm>
-  __device__ __forceinline__ void finish(const Prm& prm, const Seg& s, int lane) {
+  __device__ __forceinline__ void finish(const Prm& prm, const Seg& s, int lane, const MergeStage& stage) {
     const int g = lane >> 2, tig = lane & 3;
     const float lt0 = warp_sum_rows(l0), lt1 = warp_sum_rows(l1);
     const int h0 = 2 * tig, h1 = 2 * tig + 1;
@@ -378,11 +378,11 @@ struct MmaPath {
       }
       if constexpr (kSibParams<Prm>) {
         if (s.shared) {
-          settle_partial<ACT, G, kMaxGroup>(prm, s, rows, lane);
+          settle_partial<ACT, G, kMaxGroup>(prm, s, rows, lane, stage);
           return;
         }
       }
-      settle_partial<ACT, G, G>(prm, s, G, lane);
+      settle_partial<ACT, G, G>(prm, s, G, lane, stage);
     }
   }
 };
@@ -544,7 +544,7 @@ struct FmaPath {
   }
 
   template <class Prm>
-  __device__ __forceinline__ void finish(const Prm& prm, const Seg& s, int lane) {
+  __device__ __forceinline__ void finish(const Prm& prm, const Seg& s, int lane, const MergeStage& stage) {
     const int r = lane >> 2, qd = lane & 3;
 #pragma unroll
     for (int gg = 0; gg < G; ++gg) {
@@ -592,7 +592,7 @@ struct FmaPath {
           ml[2 * gg + 1] = l[gg];
         }
       }
-      settle_partial<ACT, G, G>(prm, s, G, lane);
+      settle_partial<ACT, G, G>(prm, s, G, lane, stage);
     }
   }
 };
@@ -648,7 +648,7 @@ __device__ __forceinline__ bool consume_segment(Path& path, const Prm& prm, cons
                                                 Producer<KV>& prod, const CUtensorMap* tmk,
                                                 const CUtensorMap* tmv, uint8_t* ring_ptr,
                                                 uint32_t ring, uint32_t bars, uint32_t& consumed,
-                                                int w, int lane) {
+                                                int w, int lane, uint32_t merge_bar, uint32_t& merge_phase) {
   using T = Tile<KV>;
   path.begin(prm, s, lane);
 #pragma unroll 1
@@ -674,7 +674,12 @@ __device__ __forceinline__ bool consume_segment(Path& path, const Prm& prm, cons
     ++consumed;
     prod.issue(prm, tmk, tmv, ring, bars, w, lane);
   }
-  path.finish(prm, s, lane);
+  // With no copy of its own in flight (its last segment), the worker's ring
+  // can stage the partial slots of a merge.
+  MergeStage stage{nullptr, 0, 0, 0, nullptr};
+  if (prod.issued == consumed) stage = MergeStage{ring_ptr, ring, T::kRingBytes / static_cast<int>(kSlotBytes),
+                                                  merge_bar, &merge_phase};
+  path.finish(prm, s, lane, stage);
   return true;
 }
 
@@ -698,10 +703,14 @@ __global__ void __launch_bounds__(kWarps * 32)
   const uint32_t bars = dev::smem_u32(smem + kWarps * T::kRingBytes) + warp * T::kStages * 8;
   int32_t* phys_s = reinterpret_cast<int32_t*>(smem + kWarps * T::kRingBytes + kWarps * T::kStages * 8) +
                     warp * T::kStages;
+  const uint32_t merge_bar =
+      dev::smem_u32(smem + kWarps * T::kRingBytes + kWarps * T::kStages * 12) + warp * 8;
+  uint32_t merge_phase = 0;
   if (lane == 0) {
     dev::tma_prefetch_desc(&tmk);
     dev::tma_prefetch_desc(&tmv);
     for (int s = 0; s < T::kStages; ++s) dev::mbar_init(bars + s * 8, 1);
+    dev::mbar_init(merge_bar, 1);
     dev::fence_mbar_init();
   }
   __syncwarp();
@@ -728,7 +737,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     const Seg s = cur.next(prm);
     if (!s.valid) break;
     const bool ok =
-        consume_segment<KV, ACT, G>(path, prm, s, prod, &tmk, &tmv, ring_ptr, ring, bars, consumed, w, lane);
+        consume_segment<KV, ACT, G>(path, prm, s, prod, &tmk, &tmv, ring_ptr, ring, bars, consumed, w, lane,
+                                    merge_bar, merge_phase);
     if (!ok) {
       failed = true;
       break;
@@ -809,8 +819,9 @@ __global__ void __launch_bounds__(128) reduce_fixed_kernel(const __grid_constant
 // ================================================================== launchers
 template <int KV>
 constexpr size_t smem_bytes() {
-  // rings, one mbarrier per stage, the physical block id of each staged block
-  return 1024 + kWarps * Tile<KV>::kRingBytes + kWarps * Tile<KV>::kStages * (8 + 4);
+  // rings, one mbarrier per stage, the cache row of each staged block, one
+  // mbarrier per warp for merge staging
+  return 1024 + kWarps * Tile<KV>::kRingBytes + kWarps * Tile<KV>::kStages * (8 + 4) + kWarps * 8;
 }
 
 template <int KV, int ACT, int G, class PlanT>
