@@ -482,7 +482,8 @@ def _run_ours(a, rank, world, local_rank, device):
     launch_ms = sum(loop_ms) / (len(loop_ms) * w.num_layers)     # per layer
     launch_bytes = sum(loop_bytes) / (len(loop_bytes) * w.num_layers)
     achieved = launch_bytes / (launch_ms * 1e-3) / 1e9
-    tr = traffic_record(f"{w.name}:decode")
+    kern = pa.pa_last_decode_kernel(r.pool)
+    tr = traffic_record(f"{w.name}:decode" + ("_tcgen05" if kern == "tcgen05" else ""))
     line = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -529,7 +530,7 @@ def _run_ours(a, rank, world, local_rank, device):
     }
     line["config"]["append"] = ("fused into the decode launch (pa_decode_attention_append)" if r.fused
                                 else "separate launch (pa_append_kv)")
-    line["config"]["decode_kernel"] = pa.pa_last_decode_kernel(r.pool)
+    line["config"]["decode_kernel"] = kern
     if w.name == "tiny":
         line["graph_batch"] = graph_batch(r, 1000)
     if rank == 0 and not a.no_cpu:
