@@ -168,6 +168,10 @@ class ClockSampler:
         self._t = None
 
     def __enter__(self):
+        # the step loop holds the interpreter between its library calls: switch
+        # threads often enough that the sampler runs every few hundred us
+        self._switch = sys.getswitchinterval()
+        sys.setswitchinterval(0.0002)
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -195,12 +199,13 @@ class ClockSampler:
                         self.reasons.add(nm)
             except Exception:
                 break
-            time.sleep(0.002)
+            time.sleep(0.0005)
 
     def __exit__(self, *a):
         self._stop.set()
         if self._t:
             self._t.join()
+        sys.setswitchinterval(self._switch)
 
     def summary(self):
         return {
@@ -521,6 +526,8 @@ def _run_ours(a, rank, world, local_rank, device):
         },
         "logical_decode_gbs": round(world * logical / (ms * 1e-3) / 1e9, 1),
         "gpu_launches": int(launches),
+        "step_loop_ms": {"min": round(min(loop_ms), 4), "median": round(statistics.median(loop_ms), 4),
+                         "max": round(max(loop_ms), 4)},
         "host_enqueue_ms_per_step": round(host_ms / a.steps, 4),
         # the first timed step starts with an empty launch queue, so its host
         # time is the enqueue cost itself; later steps can wait for queue room
