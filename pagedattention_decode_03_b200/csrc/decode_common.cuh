@@ -229,6 +229,55 @@ __device__ __forceinline__ BlockRef locate(const DecodeKParams<SibPlan>& prm, co
                   ((1u << G) - 1u) << (j * G), item};
 }
 
+// The members of a segment's unit held in registers, lane j < m holding
+// member j's item, own-block start in the unit (part), table row and length,
+// so a warp locates positions with shuffles instead of walking the plan in
+// parameter memory: a walk whose lanes look at different positions makes
+// divergent parameter loads, which the hardware serialises.  (Plain units
+// have one member and need none of this.)
+struct Members {
+  int32_t m, cp;                    // members, shared blocks at the unit's start
+  int32_t item, part, seq, len;     // member `lane` (lanes < m)
+};
+__device__ __forceinline__ Members load_members(const DecodeKParams<DecodePlan>&, const Seg& s, int) {
+  return Members{1, 0, s.i, 0, s.seq, s.len};
+}
+__device__ __forceinline__ Members load_members(const DecodeKParams<SibPlan>& prm, const Seg& s, int lane) {
+  const SibPlan& P = prm.plan;
+  const int m0 = P.mem0[s.k];
+  Members u{P.mem0[s.k + 1] - m0, P.cp[s.k], s.i, 0, s.seq, s.len};
+  if (lane < u.m) {
+    u.item = P.mem[m0 + lane];
+    u.part = P.part[u.item];
+    u.seq = P.seq[u.item];
+    u.len = P.len[u.item];
+  }
+  return u;
+}
+// locate() from registers: every lane may ask for its own position o; all 32
+// lanes must call it together.
+template <int G>
+__device__ __forceinline__ BlockRef locate_in(const DecodeKParams<DecodePlan>&, const Members&, const Seg& s,
+                                              int o) {
+  return BlockRef{s.seq, o, s.len, 0xffu, s.i};
+}
+template <int G>
+__device__ __forceinline__ BlockRef locate_in(const DecodeKParams<SibPlan>&, const Members& u, const Seg& s,
+                                              int o) {
+  int j = 0;
+#pragma unroll
+  for (int jj = 1; jj < kMaxGroup; ++jj) {
+    const int pj = __shfl_sync(0xffffffffu, u.part, jj);
+    if (jj < u.m && pj <= o) j = jj;
+  }
+  const int item = __shfl_sync(0xffffffffu, u.item, j);
+  const int part = __shfl_sync(0xffffffffu, u.part, j);
+  const int seq = __shfl_sync(0xffffffffu, u.seq, j);
+  const int len = __shfl_sync(0xffffffffu, u.len, j);
+  if (o < u.cp) return BlockRef{s.seq, o, s.len, 0xffu, s.i};
+  return BlockRef{seq, u.cp + (o - part), len, ((1u << G) - 1u) << (j * G), item};
+}
+
 // The segments of one worker, in processing order.  Stream-K: a worker's last
 // segment, when it starts inside the worker's share (the head of a sequence
 // cut at the share's end), is processed first, then the share from its start

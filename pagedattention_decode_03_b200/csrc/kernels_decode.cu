@@ -73,6 +73,7 @@ struct Producer {
   Seg seg;
   int32_t b;          // next block of seg to fetch
   int32_t tc_val, tc_base, tc_unit;
+  Members mem;        // members of seg's unit, for the table refreshes
   uint32_t issued;
   int32_t* phys_s;    // shared memory: first cache row (token slot) of each staged tile
 
@@ -82,6 +83,7 @@ struct Producer {
     cur = c;
     seg = cur.next(prm);
     b = seg.b0;
+    mem = load_members(prm, seg, threadIdx.x & 31);
     tc_unit = -1;
     tc_base = 0;
     tc_val = 0;
@@ -98,6 +100,7 @@ struct Producer {
       seg = cur.next(prm);
       if (!seg.valid) return;
       b = seg.b0;
+      mem = load_members(prm, seg, lane);
     }
     // physical ids of the unit's tiles b .. b+31, one per lane (a sibling
     // set's positions run through several table rows); the low bit of a
@@ -105,7 +108,7 @@ struct Producer {
     if (seg.k != tc_unit || b < tc_base || b >= tc_base + 32) {
       tc_unit = seg.k;
       tc_base = b;
-      const BlockRef r = locate<1>(prm, seg, b + lane);
+      const BlockRef r = locate_in<1>(prm, mem, seg, b + lane);
       const int32_t e = r.b >> prm.bshift;
       tc_val = r.b >= 0 && e < prm.mbps ? prm.tables[static_cast<int64_t>(r.seq) * prm.mbps + e] : 0;
       // physical id in the upper bits, half in bit 0 (ids < 2^30)
@@ -651,6 +654,7 @@ __device__ __forceinline__ bool consume_segment(Path& path, const Prm& prm, cons
                                                 int w, int lane, uint32_t merge_bar, uint32_t& merge_phase) {
   using T = Tile<KV>;
   path.begin(prm, s, lane);
+  const Members mem = load_members(prm, s, lane);
 #pragma unroll 1
   for (int b = s.b0; b < s.b1; ++b) {
     const uint32_t stage = consumed % T::kStages;
@@ -659,7 +663,7 @@ __device__ __forceinline__ bool consume_segment(Path& path, const Prm& prm, cons
       if (lane == 0) atomicOr(prm.err, kErrTimeout);
       return false;
     }
-    const BlockRef br = locate<G>(prm, s, b);
+    const BlockRef br = locate_in<G>(prm, mem, s, b);
     const int nvalid = max(0, min(kBlock, br.len - br.b * kBlock));
     uint8_t* st = ring_ptr + stage * T::kStageBytes;
     if (nvalid < kBlock) zero_tail_rows<KV>(st + T::kBytes, nvalid, lane);
