@@ -34,6 +34,14 @@
  *   - Sequence ids are integers in [0, max_seqs).
  *   - pa_last_error() returns a description of the last failure on the
  *     calling thread.
+ *   - Log: the environment variable PA_LOG (read once per process) set to 1
+ *     writes one "[pa] <status>: <message>" line to stderr for every failing
+ *     call; 2 adds one line per state-changing call (pool creation,
+ *     allocation, fork, free, swap, append, and each decode with the kernel
+ *     and work split it chose).  Unset, 0 or not a number: no output.
+ *   - Profiling: a library built with PA_NVTX defined (the build's --nvtx
+ *     option) opens an NVTX range named after the call around every entry
+ *     point; otherwise the ranges compile to nothing.
  *
  * Device data layout (bytes, row-major, caller-allocated):
  *   k_cache, v_cache: [num_layers][num_blocks][num_kv_heads][block_size][head_dim]

@@ -19,6 +19,7 @@
 #include "block_manager.h"
 #include "pa.h"
 #include "pa_internal.h"
+#include "trace.h"
 
 namespace {
 
@@ -26,11 +27,13 @@ thread_local std::string g_last_error;
 
 pa_status fail(pa_status st, const std::string& msg) {
   g_last_error = msg;
+  pa::logf(1, "%s: %s", pa_status_string(st), msg.c_str());
   return st;
 }
 
 pa_status cuda_fail(cudaError_t e, const char* what) {
   g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+  pa::logf(1, "%s: %s", pa_status_string(PA_ERR_CUDA), g_last_error.c_str());
   return PA_ERR_CUDA;
 }
 
@@ -84,7 +87,10 @@ struct DeviceGuard {
 }  // namespace
 
 namespace pa {
-void set_last_error(const std::string& msg) { g_last_error = msg; }
+void set_last_error(const std::string& msg) {
+  g_last_error = msg;
+  if (!msg.empty()) logf(1, "error: %s", msg.c_str());  // the caller's status is not known here
+}
 }  // namespace pa
 
 struct pa_pool {
@@ -331,6 +337,7 @@ bool build_sib_plan(const pa_pool* p, const int32_t* seqs, int32_t cnt, int grou
 extern "C" {
 
 size_t pa_workspace_size(const pa_pool_desc* d) {
+  PA_RANGE();
   if (!d || d->max_seqs <= 0 || d->max_blocks_per_seq <= 0 || d->num_kv_heads <= 0 ||
       d->block_size <= 0)
     return 0;
@@ -339,6 +346,7 @@ size_t pa_workspace_size(const pa_pool_desc* d) {
 }
 
 pa_status pa_pool_create(const pa_pool_desc* d, pa_pool** out) {
+  PA_RANGE();
   g_last_error.clear();
   if (!d || !out) return fail(PA_ERR_INVALID_ARG, "null argument");
   if (d->head_dim != pa::kHeadDim) return fail(PA_ERR_INVALID_ARG, "head_dim must be 128");
@@ -416,14 +424,21 @@ pa_status pa_pool_create(const pa_pool_desc* d, pa_pool** out) {
   v.mbps = d->max_blocks_per_seq;
   v.kv_dtype = d->kv_dtype;
   v.act_dtype = d->act_dtype;
+  pa::logf(2, "pool_create: %s, %d layers, %d blocks of %d tokens, %d KV heads, %d sequences x %d blocks, "
+           "kv dtype %d", host_only ? "host only" : "device buffers", d->num_layers, d->num_blocks,
+           d->block_size, d->num_kv_heads, d->max_seqs, d->max_blocks_per_seq, d->kv_dtype);
   *out = p.release();
   return PA_OK;
 }
 
-void pa_pool_destroy(pa_pool* p) { delete p; }
+void pa_pool_destroy(pa_pool* p) {
+  PA_RANGE();
+  delete p;
+}
 
 pa_status pa_alloc_blocks_n(pa_pool* p, int32_t n, const int32_t* seqs, const int32_t* new_lens,
                             void* stream, int32_t* n_done) {
+  PA_RANGE();
   g_last_error.clear();
   if (n_done) *n_done = 0;
   if (!p || n < 0 || (n > 0 && (!seqs || !new_lens)))
@@ -436,28 +451,35 @@ pa_status pa_alloc_blocks_n(pa_pool* p, int32_t n, const int32_t* seqs, const in
     if (st != PA_OK) break;
   }
   if (n_done) *n_done = k;
+  pa::logf(2, "alloc_blocks: %d of %d sequences reserved, %zu block copies", k, n, p->cows.size());
   const pa_status launch = launch_cows(p, static_cast<cudaStream_t>(stream));
   return st != PA_OK ? st : launch;
 }
 
 pa_status pa_alloc_blocks(pa_pool* p, int32_t seq, int32_t new_len, void* stream) {
+  PA_RANGE();
   int32_t done = 0;
   return pa_alloc_blocks_n(p, 1, &seq, &new_len, stream, &done);
 }
 
 pa_status pa_fork_cow(pa_pool* p, int32_t parent, int32_t child) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
+  pa::logf(2, "fork_cow: sequence %d -> %d", parent, child);
   return bm_status(p->bm->fork(parent, child), "pa_fork_cow");
 }
 
 pa_status pa_free(pa_pool* p, int32_t seq) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
+  pa::logf(2, "free: sequence %d", seq);
   return bm_status(p->bm->release(seq), "pa_free");
 }
 
 pa_status pa_prefix_register(pa_pool* p, int32_t seq, int32_t n_tokens, const int32_t* tokens) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p || n_tokens < 0 || (n_tokens > 0 && !tokens)) return fail(PA_ERR_INVALID_ARG, "null argument");
   pa_status st = seq_arg(p, seq);
@@ -467,6 +489,7 @@ pa_status pa_prefix_register(pa_pool* p, int32_t seq, int32_t n_tokens, const in
 
 pa_status pa_prefix_match(const pa_pool* p, int32_t n_tokens, const int32_t* tokens,
                           int32_t* n_cached) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p || !n_cached || n_tokens < 0 || (n_tokens > 0 && !tokens))
     return fail(PA_ERR_INVALID_ARG, "null argument");
@@ -476,6 +499,7 @@ pa_status pa_prefix_match(const pa_pool* p, int32_t n_tokens, const int32_t* tok
 
 pa_status pa_alloc_blocks_prefix(pa_pool* p, int32_t seq, int32_t n_tokens, const int32_t* tokens,
                                  int32_t* n_cached) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p || !n_cached || n_tokens < 0 || (n_tokens > 0 && !tokens))
     return fail(PA_ERR_INVALID_ARG, "null argument");
@@ -555,6 +579,7 @@ pa_status swap_copies(pa_pool* p, const std::vector<int32_t>& table, char* host,
 }  // namespace
 
 pa_status pa_swap_bytes(const pa_pool* p, int32_t n_tokens, size_t* bytes) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p || !bytes || n_tokens < 0) return fail(PA_ERR_INVALID_ARG, "null argument or negative length");
   *bytes = swap_image_bytes(p->d, n_tokens);
@@ -562,6 +587,7 @@ pa_status pa_swap_bytes(const pa_pool* p, int32_t n_tokens, size_t* bytes) {
 }
 
 pa_status pa_swap_out(pa_pool* p, int32_t seq, void* host, size_t host_bytes, void* stream) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
   if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
@@ -573,6 +599,7 @@ pa_status pa_swap_out(pa_pool* p, int32_t seq, void* host, size_t host_bytes, vo
   st = check_host_image(host, host_bytes, swap_image_bytes(p->d, p->bm->len(seq)));
   if (st != PA_OK) return st;
   const std::vector<int32_t> table = p->bm->table(seq);
+  pa::logf(2, "swap_out: sequence %d, %d tokens, %zu bytes", seq, p->bm->len(seq), host_bytes);
   st = swap_copies(p, table, static_cast<char*>(host), true, static_cast<cudaStream_t>(stream));
   if (st != PA_OK) return st;
   return bm_status(p->bm->release(seq), "pa_swap_out");
@@ -580,6 +607,7 @@ pa_status pa_swap_out(pa_pool* p, int32_t seq, void* host, size_t host_bytes, vo
 
 pa_status pa_swap_in(pa_pool* p, int32_t seq, int32_t n_tokens, const void* host, size_t host_bytes,
                      void* stream) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
   if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
@@ -592,6 +620,7 @@ pa_status pa_swap_in(pa_pool* p, int32_t seq, int32_t n_tokens, const void* host
   st = check_host_image(host, host_bytes, swap_image_bytes(p->d, n_tokens));
   if (st != PA_OK) return st;
   p->cows.clear();
+  pa::logf(2, "swap_in: sequence %d, %d tokens, %zu bytes", seq, n_tokens, host_bytes);
   st = bm_status(p->bm->reserve(seq, n_tokens, &p->cows), "pa_swap_in");
   if (st != PA_OK) return st;
   st = swap_copies(p, p->bm->table(seq), static_cast<char*>(const_cast<void*>(host)), false,
@@ -603,6 +632,7 @@ pa_status pa_swap_in(pa_pool* p, int32_t seq, int32_t n_tokens, const void* host
 pa_status pa_append_kv(pa_pool* p, int32_t layer, int32_t T, const int32_t* seqs,
                        const int32_t* positions, const void* k_new, const void* v_new,
                        void* stream) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
   if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
@@ -632,6 +662,7 @@ pa_status pa_append_kv(pa_pool* p, int32_t layer, int32_t T, const int32_t* seqs
   p->launches += launches;
   if (e != cudaSuccess) return cuda_fail(e, "append launch");
   md.consume(nd);
+  pa::logf(2, "append_kv: layer %d, %d rows, %d table updates", layer, T, nd);
   return PA_OK;
 }
 
@@ -764,6 +795,7 @@ pa_status decode_call(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
                    pc.seqs.size() == static_cast<size_t>(n) &&
                    std::equal(seqs, seqs + n, pc.seqs.begin());
   pa::DecodePlan& plan = pc.plan;
+  const uint64_t launches0 = p->launches;
   int32_t at = 0;
   while (at < n) {
     // Items of this launch: up to the parameter capacity, and (fixed mode) the
@@ -826,6 +858,12 @@ pa_status decode_call(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     at += cnt;
   }
+  pa::logf(2, "decode: layer %d, %d sequences, G=%d, %s kernel, %s split (%d-tile partitions), "
+           "%d sibling sets, %s, %llu launches, plan %s", layer, n, group,
+           p->last_tc ? "tcgen05" : "warp-level",
+           mode == pa::kSplitNever ? "no" : mode == pa::kSplitFixed ? "fixed" : "stream-K", part_blocks,
+           p->last_sets, k_new != nullptr ? "append fused" : "no append",
+           static_cast<unsigned long long>(p->launches - launches0), hit ? "reused" : "built");
   return PA_OK;
 }
 
@@ -834,6 +872,7 @@ pa_status decode_call(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
 pa_status pa_decode_attention(pa_pool* p, int32_t layer, int32_t n, const int32_t* seqs,
                               int32_t num_q_heads, const void* q, void* out, float scale,
                               int32_t partition_tokens, void* stream) {
+  PA_RANGE();
   g_last_error.clear();
   return decode_call(p, layer, n, seqs, num_q_heads, q, out, scale, partition_tokens, stream,
                      nullptr, nullptr);
@@ -843,6 +882,7 @@ pa_status pa_decode_attention_append(pa_pool* p, int32_t layer, int32_t n, const
                                      const void* k_new, const void* v_new, int32_t num_q_heads,
                                      const void* q, void* out, float scale,
                                      int32_t partition_tokens, void* stream) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
   if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
@@ -872,6 +912,7 @@ pa_status pa_decode_attention_append(pa_pool* p, int32_t layer, int32_t n, const
 
 pa_status pa_get_seq(pa_pool* p, int32_t seq, int32_t* len, int32_t* table, int32_t cap,
                      int32_t* nblocks) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
   pa_status st = seq_arg(p, seq);
@@ -887,6 +928,7 @@ pa_status pa_get_seq(pa_pool* p, int32_t seq, int32_t* len, int32_t* table, int3
 }
 
 pa_status pa_get_refcounts(pa_pool* p, int32_t* out, int32_t cap) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p || !out) return fail(PA_ERR_INVALID_ARG, "null argument");
   if (cap < p->d.num_blocks) return fail(PA_ERR_INVALID_ARG, "cap < num_blocks");
@@ -895,6 +937,7 @@ pa_status pa_get_refcounts(pa_pool* p, int32_t* out, int32_t cap) {
 }
 
 pa_status pa_get_free_list(pa_pool* p, int32_t* out, int32_t cap, int32_t* n) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p || !n || (cap > 0 && !out)) return fail(PA_ERR_INVALID_ARG, "null argument");
   std::vector<int32_t> fl;
@@ -906,6 +949,7 @@ pa_status pa_get_free_list(pa_pool* p, int32_t* out, int32_t cap, int32_t* n) {
 }
 
 pa_status pa_get_cached_blocks(pa_pool* p, int32_t* out, int32_t cap, int32_t* n) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p || !n || (cap > 0 && !out)) return fail(PA_ERR_INVALID_ARG, "null argument");
   std::vector<int32_t> cl;
@@ -917,6 +961,7 @@ pa_status pa_get_cached_blocks(pa_pool* p, int32_t* out, int32_t cap, int32_t* n
 }
 
 pa_status pa_get_cow_log(pa_pool* p, int32_t* pairs, int32_t cap, int32_t* n) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p || !n || (cap > 0 && !pairs)) return fail(PA_ERR_INVALID_ARG, "null argument");
   const int32_t m = std::min<int32_t>(cap, static_cast<int32_t>(p->cow_log.size()));
@@ -931,6 +976,7 @@ pa_status pa_get_cow_log(pa_pool* p, int32_t* pairs, int32_t cap, int32_t* n) {
 uint64_t pa_launch_count(const pa_pool* p) { return p ? p->launches : 0; }
 
 pa_status pa_set_decode_path(pa_pool* p, int32_t path) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
   if (path != PA_DECODE_AUTO && path != PA_DECODE_WARP && path != PA_DECODE_TCGEN05)
@@ -940,6 +986,7 @@ pa_status pa_set_decode_path(pa_pool* p, int32_t path) {
 }
 
 pa_status pa_last_decode_kernel(const pa_pool* p, int32_t* tcgen05) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p || !tcgen05) return fail(PA_ERR_INVALID_ARG, "null argument");
   *tcgen05 = p->last_tc ? 1 : 0;
@@ -948,6 +995,7 @@ pa_status pa_last_decode_kernel(const pa_pool* p, int32_t* tcgen05) {
 
 pa_status pa_plan_siblings(const pa_pool* p, int32_t n, const int32_t* seqs, int32_t group,
                            int32_t* set_of, int32_t* set_cp, int32_t* n_sets) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p || (n > 0 && (!seqs || !set_of || !set_cp)) || !n_sets)
     return fail(PA_ERR_INVALID_ARG, "null argument");
@@ -973,6 +1021,7 @@ pa_status pa_plan_siblings(const pa_pool* p, int32_t n, const int32_t* seqs, int
 }
 
 pa_status pa_check_device_errors(pa_pool* p, void* stream, uint32_t* bits) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p || !bits) return fail(PA_ERR_INVALID_ARG, "null argument");
   if (p->host_only) return fail(PA_ERR_INVALID_ARG, "host-only pool: no device buffers");
@@ -1005,6 +1054,7 @@ pa_status pa_check_device_errors(pa_pool* p, void* stream, uint32_t* bits) {
 }
 
 pa_status pa_last_decode_plan(const pa_pool* p, int32_t* shared_sets, int64_t* kv_tiles) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
   if (shared_sets) *shared_sets = p->last_sets;
@@ -1013,6 +1063,7 @@ pa_status pa_last_decode_plan(const pa_pool* p, int32_t* shared_sets, int64_t* k
 }
 
 pa_status pa_debug_fail_after(pa_pool* p, int32_t n) {
+  PA_RANGE();
   g_last_error.clear();
   if (!p) return fail(PA_ERR_INVALID_ARG, "null pool");
   p->bm->set_fail_after(n);

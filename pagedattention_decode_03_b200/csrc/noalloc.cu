@@ -29,6 +29,7 @@
 
 #include "pa.h"
 #include "pa_internal.h"
+#include "trace.h"
 
 namespace {
 
@@ -85,6 +86,7 @@ extern "C" pa_status pa_decode_attention_noalloc(const pa_pool_desc* d, int32_t 
                                                  const int32_t* seq_lens, int32_t num_q_heads,
                                                  const void* q, void* out, float scale,
                                                  void* stream) {
+  PA_RANGE();
   pa::set_last_error("");
   if (!d || !block_tables || !seq_lens || !q || !out || !d->k_cache || !d->v_cache)
     return fail(PA_ERR_INVALID_ARG, "null argument");
@@ -205,10 +207,12 @@ extern "C" pa_status pa_decode_attention_noalloc(const pa_pool_desc* d, int32_t 
   int launches = 0;
   e = pa::launch_decode(v, maps, plan, args, s, &launches);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));
+  pa::logf(2, "decode_noalloc: layer %d, %d sequences, G=%d, %d workers", layer, n, group, plan.workers);
   return PA_OK;
 }
 
 extern "C" pa_status pa_noalloc_check_errors(int32_t device, void* stream, uint32_t* bits) {
+  PA_RANGE();
   pa::set_last_error("");
   if (!bits) return fail(PA_ERR_INVALID_ARG, "null argument");
   if (device < 0 || device >= kMaxDevices) return fail(PA_ERR_INVALID_ARG, "device ordinal out of range");
