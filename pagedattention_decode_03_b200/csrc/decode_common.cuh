@@ -458,25 +458,80 @@ __device__ __forceinline__ int64_t row_offset(const Prm& prm, const Seg& s, int 
 }
 
 // One warp merges query rows 0 .. rows-1 (rows <= R) of one unit over
-// `nslots` partial slots, online: for each slot k (m_k, l_k, o~_k) the running
-// (M, L, acc) become
-//   M' = max(M, m_k), L' = L 2^(M-M') + l_k 2^(m_k-M'), acc' likewise,
-// with 0 in place of M' while every slot seen so far is empty (m = -inf, a
-// row that no token of those slots reached).
-// Slots are taken a few at a time with every load of a batch issued before
-// any use, so a typical cut sequence (2-4 partials) costs one L2 round trip.
+// `nslots` partial slots (m_k, l_k, o~_k) in two passes:
+//   M = max_k m_k (lanes split the slots, butterfly max), then in slot order
+//   w_k = 2^(m_k - M'), L = sum w_k l_k, acc = sum w_k o~_k  (M' = M, or 0 for
+//   a row that no token of any slot reached),
+// and writes acc / L.  With a fixed reference the slots' terms are
+// independent, and every row is computed (rows past `rows` hold no data and
+// are not written), so the rows' chains interleave.  The arithmetic depends
+// only on the slot order, never on how many slots are in flight, so this and
+// merge_unit_warp_staged agree bit for bit.
 // Each lane owns d = 4*lane .. 4*lane+3 of every row and reads the (m, l)
 // pairs itself (same address in all lanes: one broadcast transaction).
 // out_of(r) = element offset of output row r.
+template <int R, class SlotFn>
+__device__ __forceinline__ void merge_max_pass(const float* partials, int nslots, SlotFn slot_of, int lane,
+                                               float (&M)[R]) {
+#pragma unroll
+  for (int gg = 0; gg < R; ++gg) M[gg] = -INFINITY;
+  for (int k = lane; k < nslots; k += 32) {
+    const float* ml = partials + static_cast<int64_t>(slot_of(k)) * kPartialSlotFloats + kMaxGroup * kHeadDim;
+#pragma unroll
+    for (int gg = 0; gg < R; ++gg) M[gg] = fmaxf(M[gg], __ldcg(ml + 2 * gg));
+  }
+#pragma unroll
+  for (int gg = 0; gg < R; ++gg) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M[gg] = fmaxf(M[gg], __shfl_xor_sync(0xffffffffu, M[gg], o));
+    if (M[gg] == -INFINITY) M[gg] = 0.f;  // the reference of an empty row
+  }
+}
+
+// One slot's terms into every row's sums (reference M).
+template <int R>
+__device__ __forceinline__ void merge_add_slot(const float2 (&ml)[R], const float4 (&x)[R], const float (&M)[R],
+                                               float (&L)[R], float4 (&acc)[R]) {
+#pragma unroll
+  for (int gg = 0; gg < R; ++gg) {
+    const float w = dev::exp2_approx(ml[gg].x - M[gg]);
+    L[gg] = fmaf(ml[gg].y, w, L[gg]);
+    acc[gg].x = fmaf(x[gg].x, w, acc[gg].x);
+    acc[gg].y = fmaf(x[gg].y, w, acc[gg].y);
+    acc[gg].z = fmaf(x[gg].z, w, acc[gg].z);
+    acc[gg].w = fmaf(x[gg].w, w, acc[gg].w);
+  }
+}
+
+// acc / L of rows < rows to the output; lane r < rows holds row r's offset.
+template <int ACT, int R>
+__device__ __forceinline__ void merge_write(uint16_t* out, int rows, int64_t out_lane, const float (&L)[R],
+                                            const float4 (&acc)[R], int lane) {
+#pragma unroll
+  for (int gg = 0; gg < R; ++gg) {
+    const int64_t off = __shfl_sync(0xffffffffu, out_lane, gg);
+    if (gg < rows) {
+      const float inv = 1.f / L[gg];
+      const uint32_t a = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].x * inv)) |
+                         (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].y * inv)) << 16);
+      const uint32_t b = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].z * inv)) |
+                         (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].w * inv)) << 16);
+      *reinterpret_cast<uint2*>(out + off + 4 * lane) = make_uint2(a, b);
+    }
+  }
+}
+
+// Slots are read a few at a time, every load of a batch issued before any use.
 template <int ACT, int R, class SlotFn, class OutFn>
 __device__ __forceinline__ void merge_unit_warp(const float* partials, uint16_t* out, int nslots,
                                                 int rows, SlotFn slot_of, OutFn out_of, int lane) {
   constexpr int kBatch = R >= 8 ? 2 : (R >= 4 ? 3 : 4);  // loads in flight within the register budget
+  const int64_t out_lane = lane < rows ? out_of(lane) : 0;
   float M[R], L[R];
   float4 acc[R];
+  merge_max_pass<R>(partials, nslots, slot_of, lane, M);
 #pragma unroll
   for (int gg = 0; gg < R; ++gg) {
-    M[gg] = -INFINITY;
     L[gg] = 0.f;
     acc[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
@@ -489,45 +544,16 @@ __device__ __forceinline__ void merge_unit_warp(const float* partials, uint16_t*
         const float* slot = partials + static_cast<int64_t>(slot_of(k0 + j)) * kPartialSlotFloats;
 #pragma unroll
         for (int gg = 0; gg < R; ++gg) {
-          if (gg < rows) {
-            ml[j][gg] = __ldcg(reinterpret_cast<const float2*>(slot + kMaxGroup * kHeadDim) + gg);
-            x[j][gg] = __ldcg(reinterpret_cast<const float4*>(slot + gg * kHeadDim) + lane);
-          }
+          ml[j][gg] = __ldcg(reinterpret_cast<const float2*>(slot + kMaxGroup * kHeadDim) + gg);
+          x[j][gg] = __ldcg(reinterpret_cast<const float4*>(slot + gg * kHeadDim) + lane);
         }
       }
     }
 #pragma unroll
-    for (int j = 0; j < kBatch; ++j) {
-      if (k0 + j < nslots) {
-#pragma unroll
-        for (int gg = 0; gg < R; ++gg) {
-          if (gg < rows) {
-            const float mn = fmaxf(M[gg], ml[j][gg].x);
-            const float ref = mn == -INFINITY ? 0.f : mn;
-            const float a = dev::exp2_approx(M[gg] - ref);        // 0 on the first slot
-            const float b = dev::exp2_approx(ml[j][gg].x - ref);
-            M[gg] = mn;
-            L[gg] = L[gg] * a + ml[j][gg].y * b;
-            acc[gg].x = acc[gg].x * a + x[j][gg].x * b;
-            acc[gg].y = acc[gg].y * a + x[j][gg].y * b;
-            acc[gg].z = acc[gg].z * a + x[j][gg].z * b;
-            acc[gg].w = acc[gg].w * a + x[j][gg].w * b;
-          }
-        }
-      }
-    }
+    for (int j = 0; j < kBatch; ++j)
+      if (k0 + j < nslots) merge_add_slot<R>(ml[j], x[j], M, L, acc);
   }
-#pragma unroll
-  for (int gg = 0; gg < R; ++gg) {
-    if (gg < rows) {
-      const float inv = 1.f / L[gg];
-      const uint32_t a = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].x * inv)) |
-                         (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].y * inv)) << 16);
-      const uint32_t b = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].z * inv)) |
-                         (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].w * inv)) << 16);
-      *reinterpret_cast<uint2*>(out + out_of(gg) + 4 * lane) = make_uint2(a, b);
-    }
-  }
+  merge_write<ACT, R>(out, rows, out_lane, L, acc, lane);
 }
 
 __device__ __forceinline__ int atom_add_acq_rel(int32_t* p, int32_t v) {
@@ -549,33 +575,40 @@ struct MergeStage {
 constexpr uint32_t kSlotBytes = sizeof(float) * kPartialSlotFloats;
 
 // merge_unit_warp with the slots brought into shared memory by bulk copies,
-// stage.slots at a time (one copy per slot, all in flight together), so a
-// merge of n slots takes ceil(n / stage.slots) round trips to L2 instead of
-// one per two slots.  Same arithmetic, same slot order, so the same result
-// bit for bit.  False if a copy wait gave up (nothing was written).
+// stage.slots at a time (one copy per slot, all in flight together, the first
+// round's copies overlapping the maximum pass), so a merge of n slots takes
+// ceil(n / stage.slots) round trips to L2 instead of one per two slots.  Same
+// arithmetic, same slot order, so the same result bit for bit.  False if a
+// copy wait gave up (nothing was written).
 template <int ACT, int R, class SlotFn, class OutFn>
 __device__ __forceinline__ bool merge_unit_warp_staged(const float* partials, uint16_t* out, int nslots,
                                                        int rows, SlotFn slot_of, OutFn out_of, int lane,
                                                        const MergeStage& st) {
-  float M[R], L[R];
-  float4 acc[R];
-#pragma unroll
-  for (int gg = 0; gg < R; ++gg) {
-    M[gg] = -INFINITY;
-    L[gg] = 0.f;
-    acc[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+  const int64_t out_lane = lane < rows ? out_of(lane) : 0;
   // the arrivals' acquire comes before the copies' reads; the ring's last
   // reads come before the copies' writes
   dev::fence_proxy_async_global();
   dev::fence_proxy_async_smem();
-  for (int k0 = 0; k0 < nslots; k0 += st.slots) {
+  auto issue = [&](int k0) {
     const int cnt = min(st.slots, nslots - k0);
     if (lane == 0) dev::mbar_arrive_expect_tx(st.bar, cnt * kSlotBytes);
     __syncwarp();
     if (lane < cnt)
       dev::bulk_load(st.addr + lane * kSlotBytes,
                      partials + static_cast<int64_t>(slot_of(k0 + lane)) * kPartialSlotFloats, kSlotBytes, st.bar);
+  };
+  issue(0);
+  float M[R], L[R];
+  float4 acc[R];
+  merge_max_pass<R>(partials, nslots, slot_of, lane, M);
+#pragma unroll
+  for (int gg = 0; gg < R; ++gg) {
+    L[gg] = 0.f;
+    acc[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int k0 = 0; k0 < nslots; k0 += st.slots) {
+    if (k0 > 0) issue(k0);
+    const int cnt = min(st.slots, nslots - k0);
     const bool ok = dev::mbar_wait_bounded(st.bar, *st.phase & 1u, kWaitLimit);
     if (!__all_sync(0xffffffffu, ok)) {
       // let the copies land before the ring can be reused or released
@@ -586,38 +619,19 @@ __device__ __forceinline__ bool merge_unit_warp_staged(const float* partials, ui
     ++*st.phase;
     for (int j = 0; j < cnt; ++j) {
       const float* slot = reinterpret_cast<const float*>(st.ptr + j * kSlotBytes);
+      float2 ml[R];
+      float4 x[R];
 #pragma unroll
       for (int gg = 0; gg < R; ++gg) {
-        if (gg < rows) {
-          const float2 ml = *reinterpret_cast<const float2*>(slot + kMaxGroup * kHeadDim + 2 * gg);
-          const float4 x = *reinterpret_cast<const float4*>(slot + gg * kHeadDim + 4 * lane);
-          const float mn = fmaxf(M[gg], ml.x);
-          const float ref = mn == -INFINITY ? 0.f : mn;
-          const float a = dev::exp2_approx(M[gg] - ref);
-          const float b = dev::exp2_approx(ml.x - ref);
-          M[gg] = mn;
-          L[gg] = L[gg] * a + ml.y * b;
-          acc[gg].x = acc[gg].x * a + x.x * b;
-          acc[gg].y = acc[gg].y * a + x.y * b;
-          acc[gg].z = acc[gg].z * a + x.z * b;
-          acc[gg].w = acc[gg].w * a + x.w * b;
-        }
+        ml[gg] = *reinterpret_cast<const float2*>(slot + kMaxGroup * kHeadDim + 2 * gg);
+        x[gg] = *reinterpret_cast<const float4*>(slot + gg * kHeadDim + 4 * lane);
       }
+      merge_add_slot<R>(ml, x, M, L, acc);
     }
     __syncwarp();  // every lane is done with the stage before it is refilled
     dev::fence_proxy_async_smem();
   }
-#pragma unroll
-  for (int gg = 0; gg < R; ++gg) {
-    if (gg < rows) {
-      const float inv = 1.f / L[gg];
-      const uint32_t a = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].x * inv)) |
-                         (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].y * inv)) << 16);
-      const uint32_t b = static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].z * inv)) |
-                         (static_cast<uint32_t>(f32_to_act<ACT>(acc[gg].w * inv)) << 16);
-      *reinterpret_cast<uint2*>(out + out_of(gg) + 4 * lane) = make_uint2(a, b);
-    }
-  }
+  merge_write<ACT, R>(out, rows, out_lane, L, acc, lane);
   return true;
 }
 

@@ -206,8 +206,9 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 // the kernel before it in the stream is still running.  Before its first
 // access to memory that earlier work may write or read, it waits for that
 // work to finish and become visible (returns at once when there is no
-// programmatic dependency); after that it lets the next such kernel start
-// its own prologue.
+// programmatic dependency).  grid_dep_launch lets the next such kernel start
+// placing its blocks; the short kernels signal right after their wait, the
+// decode kernels once their last copy is issued.
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

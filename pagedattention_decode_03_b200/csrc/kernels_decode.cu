@@ -98,7 +98,14 @@ struct Producer {
     if (!seg.valid) return;
     if (b == seg.b1) {
       seg = cur.next(prm);
-      if (!seg.valid) return;
+      if (!seg.valid) {
+        // every copy of this worker is out: let the next kernel in the stream
+        // start placing its blocks.  (Signalled at kernel start instead, the
+        // queued successor's launch slowed this kernel's first copies from
+        // ~1.6 to ~4.5 us in traces of back-to-back layers.)
+        dev::grid_dep_launch();
+        return;
+      }
       b = seg.b0;
       mem = load_members(prm, seg, lane);
     }
@@ -727,7 +734,6 @@ __global__ void __launch_bounds__(kWarps * 32)
   cur.init(prm, g0, g1, w);  // kernel parameters only: may overlap the previous kernel
   prod.init(prm, cur);
   dev::grid_dep_wait();
-  dev::grid_dep_launch();
 #pragma unroll 1
   for (int k = 0; k < T::kStages; ++k) prod.issue(prm, &tmk, &tmv, ring, bars, w, lane);
 

@@ -250,7 +250,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   Cursor cur;
   cur.init(prm, g0, g1, w);  // kernel parameters only: may overlap the previous kernel
   dev::grid_dep_wait();
-  dev::grid_dep_launch();
   bool failed = false;
 
   if (warp == 0) {
@@ -316,6 +315,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (failed) break;
       ++seg_i;
     }
+    // every copy is out: the next kernel in the stream may start placing its
+    // blocks (not at kernel start: a queued successor's launch slows the
+    // first copies)
+    dev::grid_dep_launch();
     // let every copy already issued land before the CTA can exit: the last
     // tile of each stage and the last load of each Q buffer
     for (uint32_t k = tile_i > kTcStages ? tile_i - kTcStages : 0; k < tile_i; ++k)
