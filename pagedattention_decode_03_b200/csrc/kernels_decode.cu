@@ -90,6 +90,32 @@ struct Producer {
     issued = 0;
   }
 
+  // Before the dependency wait: prefetch the first n tiles of the first
+  // segment into L2, while the previous kernel's tail leaves HBM mostly idle.
+  // The table entries may be stale here (a kernel still running may rewrite
+  // them): a stale id only wastes a prefetch, since the copies after the wait
+  // read the tables again and L2 holds the current data; ids are clamped into
+  // the pool, so every address lies inside the cache.
+  template <class Prm>
+  __device__ __forceinline__ void prefetch_l2(const Prm& prm, int n, int lane) {
+    if (!seg.valid) return;  // warp-uniform
+    const int nb = min(n, seg.b1 - seg.b0);
+    if (nb <= 0) return;     // warp-uniform
+    // locate_in is collective (shuffles over a unit's members): all lanes
+    const BlockRef r = locate_in<1>(prm, mem, seg, seg.b0 + min(lane, nb - 1));
+    if (lane >= nb) return;
+    const int32_t e = r.b >> prm.bshift;
+    int32_t phys = r.b >= 0 && e < prm.mbps ? prm.tables[static_cast<int64_t>(r.seq) * prm.mbps + e] : 0;
+    if (static_cast<uint32_t>(phys) >= static_cast<uint32_t>(prm.num_blocks)) phys = 0;
+    const int64_t row =
+        ((static_cast<int64_t>(prm.layer) * prm.num_blocks + phys) * prm.num_kv_heads + seg.h) *
+            (kBlock << prm.bshift) +
+        (r.b & ((1 << prm.bshift) - 1)) * kBlock;
+    const int64_t off = row * kHeadDim * (KV == kFP8 ? 1 : 2);
+    dev::bulk_prefetch_l2(prm.k_cache + off, Tile<KV>::kBytes);
+    dev::bulk_prefetch_l2(prm.v_cache + off, Tile<KV>::kBytes);
+  }
+
   // Fetch the next block of this worker into stage issued % kStages.
   template <class Prm>
   __device__ __forceinline__ void issue(const Prm& prm, const CUtensorMap* tmk,
@@ -733,6 +759,12 @@ __global__ void __launch_bounds__(kWarps * 32)
   Cursor cur;
   cur.init(prm, g0, g1, w);  // kernel parameters only: may overlap the previous kernel
   prod.init(prm, cur);
+  // Twice the ring's depth of 16-bit tiles (measured best on the 80-layer
+  // GQA layers: 33.1 us per layer against 34.9 without, worse at 16 tiles).
+  // Not for FP8 pools, whose deeper ring covers as many tiles, nor for
+  // sibling plans, whose prologue overlaps the append launch (both measured
+  // slightly slower with it).
+  if constexpr (!kIsSib<PlanT> && KV != kFP8) prod.prefetch_l2(prm, 2 * T::kStages, lane);
   dev::grid_dep_wait();
 #pragma unroll 1
   for (int k = 0; k < T::kStages; ++k) prod.issue(prm, &tmk, &tmv, ring, bars, w, lane);
