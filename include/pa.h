@@ -27,6 +27,13 @@
  *     as void*; NULL means the legacy default stream.  The pool's device
  *     metadata is updated in stream order: calls on one pool that use
  *     different streams must be ordered by the caller.
+ *   - Kernels are launched with programmatic stream serialization (except
+ *     on the legacy default stream): a launch may start its prologue while
+ *     the previous kernel on the stream finishes, and waits for that kernel
+ *     before it reads or writes anything earlier work may touch.  The one
+ *     exception is a decode launch's L2 prefetch hints for its first cache
+ *     tiles, which cannot change any result (the data is read again after
+ *     the wait; L2 is coherent with every write).
  *   - The caller owns every device buffer (caches, scales, workspace,
  *     q / out / k_new / v_new) and keeps it alive while work that uses it is
  *     in flight.  The pool owns only host memory.
