@@ -316,6 +316,36 @@ pa_status pa_swap_out(pa_pool *pool, int32_t seq, void *host, size_t host_bytes,
 pa_status pa_swap_in(pa_pool *pool, int32_t seq, int32_t n_tokens, const void *host,
                      size_t host_bytes, void *stream);
 
+/* ---- host state checkpoint -------------------------------------------
+ * The block manager's whole host state as a byte image: the free list in
+ * order, every block's reference count, every sequence's length and block
+ * table, and the prefix cache (its index and the least-recently-used order
+ * of idle cached blocks).  pa_state_load restores it into a pool of the same
+ * geometry (num_blocks, block_size, max_seqs, max_blocks_per_seq): from then
+ * on the pool hands out, shares, copies, evicts and releases blocks exactly
+ * as the saved pool would have, and the device copy of the tables is
+ * rewritten with the next kernel launch on the pool.  The KV cache contents
+ * are the caller's buffers: a pool created over the same cache buffers and
+ * restored from the image decodes as the saved pool did.  The image is plain
+ * native-endian int32 words; it carries no device state and no copy-on-write
+ * log (pa_get_cow_log is empty after a load). */
+
+/* Bytes of the current state image. */
+pa_status pa_state_size(const pa_pool *pool, size_t *bytes);
+
+/* Write the state image to buf (cap bytes); *written = its size.
+ * Errors: PA_ERR_INVALID_ARG (null argument, cap smaller than
+ * pa_state_size). */
+pa_status pa_state_save(const pa_pool *pool, void *buf, size_t cap, size_t *written);
+
+/* Replace the pool's host state by the image in buf.  The whole image is
+ * validated first: geometry, every id in range, and a consistent pool (each
+ * block exactly one of free, referenced by the tables it appears in, or idle
+ * and cached; reference counts equal to those appearances).
+ * Errors: PA_ERR_INVALID_ARG (null argument, a truncated, corrupt or
+ * inconsistent image, another geometry); on error nothing changes. */
+pa_status pa_state_load(pa_pool *pool, const void *buf, size_t bytes);
+
 /* ---- block-granular prefix cache ([PAS] Beyond paging: radix trees and
  * continuous batching; [MKV] Block Tables and Sharing, Answer Key item 4) ----
  *

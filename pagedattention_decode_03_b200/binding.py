@@ -42,6 +42,7 @@ EXPORTS = (
     "pa_plan_siblings", "pa_prefix_register", "pa_prefix_match", "pa_alloc_blocks_prefix",
     "pa_get_cached_blocks", "pa_swap_bytes", "pa_swap_out", "pa_swap_in",
     "pa_noalloc_check_errors", "pa_set_decode_path", "pa_last_decode_kernel",
+    "pa_state_size", "pa_state_save", "pa_state_load",
 )
 
 
@@ -128,6 +129,9 @@ def lib() -> ctypes.CDLL:
         L.pa_plan_siblings.argtypes = [vp, i32, _i32p, i32, _i32p, _i32p, _i32p]
         L.pa_check_device_errors.argtypes = [vp, vp, u32p]
         L.pa_debug_fail_after.argtypes = [vp, i32]
+        L.pa_state_size.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t)]
+        L.pa_state_save.argtypes = [vp, vp, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t)]
+        L.pa_state_load.argtypes = [vp, vp, ctypes.c_size_t]
         L.pa_last_error.argtypes = []
         L.pa_last_error.restype = ctypes.c_char_p
         L.pa_status_string.argtypes = [i32]
@@ -525,3 +529,22 @@ def pa_noalloc_check_errors(device: int = 0, stream=None) -> int:
 
 def pa_debug_fail_after(pool: Pool, n: int) -> None:
     _check(lib().pa_debug_fail_after(pool.handle, n), "pa_debug_fail_after")
+
+
+def pa_state_size(pool: Pool) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().pa_state_size(pool.handle, ctypes.byref(n)), "pa_state_size")
+    return int(n.value)
+
+
+def pa_state_save(pool: Pool) -> bytes:
+    """The pool's host state image (pa.h: host state checkpoint)."""
+    buf = ctypes.create_string_buffer(pa_state_size(pool))
+    n = ctypes.c_size_t()
+    _check(lib().pa_state_save(pool.handle, buf, len(buf), ctypes.byref(n)), "pa_state_save")
+    return buf.raw[: n.value]
+
+
+def pa_state_load(pool: Pool, image: bytes) -> None:
+    buf = ctypes.create_string_buffer(bytes(image), len(image))
+    _check(lib().pa_state_load(pool.handle, buf, len(image)), "pa_state_load")

@@ -1062,6 +1062,46 @@ pa_status pa_last_decode_plan(const pa_pool* p, int32_t* shared_sets, int64_t* k
   return PA_OK;
 }
 
+pa_status pa_state_size(const pa_pool* p, size_t* bytes) {
+  PA_RANGE();
+  g_last_error.clear();
+  if (!p || !bytes) return fail(PA_ERR_INVALID_ARG, "null argument");
+  std::vector<int32_t> w;
+  p->bm->save_state(&w);
+  *bytes = w.size() * sizeof(int32_t);
+  return PA_OK;
+}
+
+pa_status pa_state_save(const pa_pool* p, void* buf, size_t cap, size_t* written) {
+  PA_RANGE();
+  g_last_error.clear();
+  if (!p || !buf || !written) return fail(PA_ERR_INVALID_ARG, "null argument");
+  std::vector<int32_t> w;
+  p->bm->save_state(&w);
+  const size_t bytes = w.size() * sizeof(int32_t);
+  if (cap < bytes) return fail(PA_ERR_INVALID_ARG, "pa_state_save: buffer smaller than pa_state_size");
+  std::memcpy(buf, w.data(), bytes);
+  *written = bytes;
+  return PA_OK;
+}
+
+pa_status pa_state_load(pa_pool* p, const void* buf, size_t bytes) {
+  PA_RANGE();
+  g_last_error.clear();
+  if (!p || (!buf && bytes > 0)) return fail(PA_ERR_INVALID_ARG, "null argument");
+  if (bytes % sizeof(int32_t) != 0) return fail(PA_ERR_INVALID_ARG, "pa_state_load: not a state image");
+  std::vector<int32_t> w(bytes / sizeof(int32_t));
+  if (bytes > 0) std::memcpy(w.data(), buf, bytes);
+  if (p->bm->load_state(w.data(), w.size()) != pa::kOk)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_state_load: not a consistent state image of a pool with this geometry");
+  p->cow_log.clear();
+  p->cows.clear();
+  p->cache.valid = false;
+  pa::logf(2, "state_load: %zu bytes", bytes);
+  return PA_OK;
+}
+
 pa_status pa_debug_fail_after(pa_pool* p, int32_t n) {
   PA_RANGE();
   g_last_error.clear();

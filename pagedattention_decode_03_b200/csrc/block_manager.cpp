@@ -383,4 +383,156 @@ void BlockManager::free_list(std::vector<int32_t>* out) const {
   }
 }
 
+
+// ------------------------------------------------------------ state image
+// int32 words:
+//   magic, num_blocks, block_size, max_seqs, max_blocks_per_seq,
+//   free count, the free blocks from the head,
+//   ref[num_blocks], block_node[num_blocks],
+//   per sequence: active, len, table size, table entries,
+//   node count N, per node: parent, block, children, key low, key high;
+//   then N * block_size tokens,
+//   spare-node count, the spare nodes (last one reused first),
+//   cached count, the idle cached blocks least recently used first.
+constexpr int32_t kStateMagic = 0x50414231;
+
+void BlockManager::save_state(std::vector<int32_t>* out) const {
+  std::vector<int32_t>& o = *out;
+  o.clear();
+  o.insert(o.end(), {kStateMagic, num_blocks_, block_size_, max_seqs_, mbps_});
+  std::vector<int32_t> fl;
+  free_list(&fl);
+  o.push_back(free_count_);
+  o.insert(o.end(), fl.begin(), fl.end());
+  o.insert(o.end(), ref_.begin(), ref_.end());
+  o.insert(o.end(), block_node_.begin(), block_node_.end());
+  for (const Seq& q : seqs_) {
+    o.push_back(q.active ? 1 : 0);
+    o.push_back(q.len);
+    o.push_back(static_cast<int32_t>(q.table.size()));
+    o.insert(o.end(), q.table.begin(), q.table.end());
+  }
+  o.push_back(static_cast<int32_t>(nodes_.size()));
+  for (const Node& nd : nodes_) {
+    o.insert(o.end(), {nd.parent, nd.block, nd.children, static_cast<int32_t>(nd.key & 0xffffffffu),
+                       static_cast<int32_t>(nd.key >> 32)});
+  }
+  o.insert(o.end(), node_tokens_.begin(), node_tokens_.end());
+  o.push_back(static_cast<int32_t>(spare_nodes_.size()));
+  o.insert(o.end(), spare_nodes_.begin(), spare_nodes_.end());
+  std::vector<int32_t> cached;
+  cached_list(&cached);
+  o.push_back(static_cast<int32_t>(cached.size()));
+  o.insert(o.end(), cached.begin(), cached.end());
+}
+
+Status BlockManager::load_state(const int32_t* w, size_t n) {
+  size_t at = 0;
+  auto take = [&](int32_t* v) {
+    if (at >= n) return false;
+    *v = w[at++];
+    return true;
+  };
+  auto in = [](int32_t v, int32_t lo, int32_t hi) { return v >= lo && v < hi; };
+  int32_t head[5];
+  for (int32_t& h : head)
+    if (!take(&h)) return kInvalidArg;
+  if (head[0] != kStateMagic || head[1] != num_blocks_ || head[2] != block_size_ || head[3] != max_seqs_ ||
+      head[4] != mbps_)
+    return kInvalidArg;
+  const int32_t NB = num_blocks_;
+  int32_t fc = 0;
+  if (!take(&fc) || !in(fc, 0, NB + 1)) return kInvalidArg;
+  std::vector<int32_t> fl(fc), ref(NB), bnode(NB);
+  std::vector<char> seen(NB, 0);
+  for (int32_t& b : fl)
+    if (!take(&b) || !in(b, 0, NB) || seen[b]++) return kInvalidArg;
+  for (int32_t& r : ref)
+    if (!take(&r) || r < 0) return kInvalidArg;
+  for (int32_t& x : bnode)
+    if (!take(&x)) return kInvalidArg;
+  std::vector<Seq> seqs(max_seqs_);
+  std::vector<int32_t> counted(NB, 0);
+  for (Seq& q : seqs) {
+    int32_t act = 0, len = 0, nt = 0;
+    if (!take(&act) || !take(&len) || !take(&nt) || !in(act, 0, 2) || !in(nt, 0, mbps_ + 1)) return kInvalidArg;
+    if (len < 0 || static_cast<int64_t>(len) > static_cast<int64_t>(mbps_) * block_size_) return kInvalidArg;
+    if (nt != (act ? (len + block_size_ - 1) / block_size_ : 0)) return kInvalidArg;
+    q.active = act != 0;
+    q.len = act ? len : 0;
+    q.table.resize(nt);
+    for (int32_t& b : q.table) {
+      if (!take(&b) || !in(b, 0, NB)) return kInvalidArg;
+      ++counted[b];
+    }
+  }
+  int32_t nn = 0;
+  if (!take(&nn) || nn < 0 || static_cast<size_t>(nn) * (5 + block_size_) > n) return kInvalidArg;
+  std::vector<Node> nodes(nn);
+  for (Node& nd : nodes) {
+    int32_t lo = 0, hi = 0;
+    if (!take(&nd.parent) || !take(&nd.block) || !take(&nd.children) || !take(&lo) || !take(&hi))
+      return kInvalidArg;
+    if (!in(nd.parent, -1, nn) || !in(nd.block, -1, NB) || nd.children < 0) return kInvalidArg;
+    nd.key = static_cast<uint64_t>(static_cast<uint32_t>(lo)) | (static_cast<uint64_t>(static_cast<uint32_t>(hi)) << 32);
+  }
+  std::vector<int32_t> toks(static_cast<size_t>(nn) * block_size_);
+  for (int32_t& t : toks)
+    if (!take(&t)) return kInvalidArg;
+  int32_t ns = 0;
+  if (!take(&ns) || !in(ns, 0, nn + 1)) return kInvalidArg;
+  std::vector<int32_t> spare(ns);
+  std::vector<char> dead(nn, 0);
+  for (int32_t& x : spare)
+    if (!take(&x) || !in(x, 0, nn) || dead[x]++) return kInvalidArg;
+  int32_t nc = 0;
+  if (!take(&nc) || !in(nc, 0, NB + 1)) return kInvalidArg;
+  std::vector<int32_t> lru(nc);
+  std::vector<char> cached(NB, 0);
+  for (int32_t& b : lru)
+    if (!take(&b) || !in(b, 0, NB) || cached[b]++) return kInvalidArg;
+  if (at != n) return kInvalidArg;
+  // consistency: every block free, referenced (its count = the tables it is
+  // in), or idle, registered and cached; live nodes and blocks name each other
+  for (int32_t b = 0; b < NB; ++b) {
+    if (ref[b] != counted[b]) return kInvalidArg;
+    if (!in(bnode[b], -1, nn) || (bnode[b] >= 0 && (dead[bnode[b]] || nodes[bnode[b]].block != b)))
+      return kInvalidArg;
+    const int kinds = (seen[b] ? 1 : 0) + (ref[b] > 0 ? 1 : 0) + (cached[b] ? 1 : 0);
+    if (kinds != 1 || (cached[b] && bnode[b] < 0) || (seen[b] && bnode[b] >= 0)) return kInvalidArg;
+  }
+  for (int32_t c = 0; c < nn; ++c)
+    if (!dead[c] && nodes[c].block >= 0 && bnode[nodes[c].block] != c) return kInvalidArg;
+
+  // apply
+  std::fill(ring_.begin(), ring_.end(), 0);
+  std::copy(fl.begin(), fl.end(), ring_.begin());
+  head_ = 0;
+  free_count_ = fc;
+  ref_.swap(ref);
+  block_node_.swap(bnode);
+  seqs_.swap(seqs);
+  nodes_.swap(nodes);
+  node_tokens_.swap(toks);
+  spare_nodes_.swap(spare);
+  index_ = NodeIndex();
+  for (int32_t c = 0; c < nn; ++c)
+    if (!dead[c]) index_.insert(nodes_[c].key, c);
+  std::fill(lru_prev_.begin(), lru_prev_.end(), -2);
+  std::fill(lru_next_.begin(), lru_next_.end(), -2);
+  lru_head_ = lru_tail_ = -1;
+  lru_count_ = 0;
+  for (int32_t b : lru) lru_push_back(b);
+  fail_after_ = -1;
+  deltas_.reset(static_cast<int64_t>(max_seqs_) * mbps_ + max_seqs_);
+  for (int32_t q = 0; q < max_seqs_; ++q) {
+    const Seq& sq = seqs_[q];
+    for (size_t j = 0; j < sq.table.size(); ++j)
+      deltas_.set(static_cast<int64_t>(q) * mbps_ + static_cast<int64_t>(j), sq.table[j]);
+    deltas_.set(static_cast<int64_t>(max_seqs_) * mbps_ + q, sq.len);
+  }
+  ++version_;
+  return kOk;
+}
+
 }  // namespace pa

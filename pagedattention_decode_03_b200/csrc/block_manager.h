@@ -137,6 +137,16 @@ class BlockManager {
   int32_t free_count() const { return free_count_; }
   void free_list(std::vector<int32_t>* out) const;
 
+  // The whole host state as int32 words (layout in block_manager.cpp), and
+  // its restore into a manager of the same geometry.  load_state validates
+  // the image completely first (ranges, and that every block is exactly one
+  // of free, referenced by the tables it sits in, or idle and cached) and
+  // changes nothing when it fails.  After a load the manager behaves exactly
+  // as the saved one did from the save on, and every table entry and length
+  // is queued for the device mirror.
+  void save_state(std::vector<int32_t>* out) const;
+  Status load_state(const int32_t* words, size_t n);
+
   void set_fail_after(int64_t n) { fail_after_ = n; }
   MirrorDeltas& deltas() { return deltas_; }
 
