@@ -538,6 +538,7 @@ def _run_ours(a, rank, world, local_rank, device):
         "vs_baseline": None,
         "dtype": w.kv_dtype if w.kv_dtype != "fp8_e4m3" else "fp8_e4m3 KV / bf16 act",
         "data": "synthetic (seeded N(0,1) K/V/Q, seeded lengths and block placement)",
+        "device": torch.cuda.get_device_name(device),
         "config": {**describe(w, partition), "parallelism": f"replicas x{world} (no exchange step)"},
         "roofline": {
             "kernel": ("decode attention" + (" with the step's append fused" if r.fused else
