@@ -2,10 +2,11 @@
  * host-only pool (no GPU) through reservation, fork, prefix reuse (the
  * 103-token prompt that reuses 96 tokens with 16-token blocks,
  * kv-cache-pagedattention-serving, Beyond paging: radix trees and continuous
- * batching), the cached list, swap sizing and error reporting, and prints
- * "ok" when every check holds. */
+ * batching), the cached list, a host state checkpoint and restore, swap
+ * sizing and error reporting, and prints "ok" when every check holds. */
 #include <stdint.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "pa.h"
@@ -59,6 +60,26 @@ int main(void) {
   int32_t idle[64], nidle = 0;
   EXPECT(pa_get_cached_blocks(p, idle, 64, &nidle) == PA_OK && nidle == 6);
   EXPECT(idle[0] == t0[5] && idle[5] == t0[0]); /* longer prefixes leave first */
+
+  /* host state checkpoint: save, change, restore */
+  size_t img = 0, wrote = 0;
+  EXPECT(pa_state_size(p, &img) == PA_OK && img > 0 && img % 4 == 0);
+  void *buf = malloc(img);
+  EXPECT(buf != NULL);
+  if (!buf) return 1;
+  EXPECT(pa_state_save(p, buf, img - 4, &wrote) == PA_ERR_INVALID_ARG); /* too small */
+  EXPECT(pa_state_save(p, buf, img, &wrote) == PA_OK && wrote == img);
+  int32_t free_before[64], nfree_before = 0, free_after[64], nfree_after = 0;
+  EXPECT(pa_get_free_list(p, free_before, 64, &nfree_before) == PA_OK);
+  EXPECT(pa_alloc_blocks(p, 3, 200, NULL) == PA_OK); /* 13 blocks */
+  EXPECT(pa_state_load(p, buf, img - 4) == PA_ERR_INVALID_ARG); /* truncated: nothing changes */
+  EXPECT(pa_get_seq(p, 3, &len, t0, 16, &nblocks) == PA_OK && len == 200);
+  EXPECT(pa_state_load(p, buf, img) == PA_OK);
+  EXPECT(pa_get_seq(p, 3, &len, t0, 16, &nblocks) == PA_ERR_NO_SEQ);
+  EXPECT(pa_get_free_list(p, free_after, 64, &nfree_after) == PA_OK && nfree_after == nfree_before &&
+         memcmp(free_before, free_after, sizeof(int32_t) * (size_t)nfree_before) == 0);
+  EXPECT(pa_get_cached_blocks(p, idle, 64, &nidle) == PA_OK && nidle == 6);
+  free(buf);
 
   size_t bytes = 0;
   EXPECT(pa_swap_bytes(p, 1525, &bytes) == PA_OK && bytes == (size_t)503316480);
