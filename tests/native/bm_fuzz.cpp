@@ -6,7 +6,10 @@
 // blocks are registered and unreferenced; a match never exceeds the prompt's
 // whole blocks and its blocks equal those the new sequence receives.  Before
 // that, the prefix index's open-addressing table runs against a std::multimap
-// with keys crowded onto three home slots.
+// with keys crowded onto three home slots.  Every 250 operations the state
+// image is saved and loaded into a fresh manager, which must show the same
+// state, and corrupted copies of the image (random words, truncations) must
+// either load into a consistent state or be refused with nothing changed.
 #include <algorithm>
 #include <cstdio>
 #include <cstdlib>
@@ -54,6 +57,53 @@ void check(const pa::BlockManager& bm) {
   for (int b = 0; b < nb; ++b) {
     CHECK(refs[b] == bm.refcount(b));
     CHECK(seen[b] == (refs[b] == 0 ? 1 : 0));
+  }
+}
+
+bool same_state(const pa::BlockManager& a, const pa::BlockManager& b) {
+  if (a.num_blocks() != b.num_blocks() || a.max_seqs() != b.max_seqs()) return false;
+  for (int s = 0; s < a.max_seqs(); ++s) {
+    if (a.active(s) != b.active(s)) return false;
+    if (a.active(s) && (a.len(s) != b.len(s) || a.table(s) != b.table(s))) return false;
+  }
+  for (int k = 0; k < a.num_blocks(); ++k)
+    if (a.refcount(k) != b.refcount(k) || a.registered(k) != b.registered(k)) return false;
+  std::vector<int32_t> fa, fb, ca, cb;
+  a.free_list(&fa);
+  b.free_list(&fb);
+  a.cached_list(&ca);
+  b.cached_list(&cb);
+  return fa == fb && ca == cb;
+}
+
+// The state image: restored into a fresh manager it gives the same state;
+// corrupted, it loads into a consistent state or changes nothing.
+void fuzz_state(const pa::BlockManager& bm, const std::vector<int32_t>& order, std::mt19937& g) {
+  std::vector<int32_t> img;
+  bm.save_state(&img);
+  pa::BlockManager r(bm.num_blocks(), bm.block_size(), bm.max_seqs(), bm.max_blocks_per_seq(), order.data());
+  CHECK(r.load_state(img.data(), img.size()) == pa::kOk);
+  CHECK(same_state(r, bm));
+  check(r);
+  for (int t = 0; t < 40 && fails == 0; ++t) {
+    std::vector<int32_t> bad = img;
+    const int flips = 1 + static_cast<int>(g() % 3);
+    for (int f = 0; f < flips; ++f) {
+      const size_t at = g() % bad.size();
+      switch (g() % 4) {
+        case 0: bad[at] = static_cast<int32_t>(g()); break;
+        case 1: bad[at] += 1; break;
+        case 2: bad[at] = -1; break;
+        default: bad.resize(at); break;
+      }
+      if (bad.empty()) break;
+    }
+    pa::BlockManager before = r;
+    if (r.load_state(bad.data(), bad.size()) == pa::kOk) {
+      check(r);
+    } else {
+      CHECK(same_state(r, before));
+    }
   }
 }
 
@@ -146,6 +196,7 @@ int main(int argc, char** argv) {
         CHECK((st == pa::kSharedBlock) == (bm.refcount(b) > 1 || bm.registered(b)));
       }
       check(bm);
+      if (it % 250 == 249) fuzz_state(bm, order, g);
     }
   }
   if (fails) return 1;

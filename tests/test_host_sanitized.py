@@ -3,7 +3,9 @@ prefix trie with its open-addressing index, cached list) under
 AddressSanitizer and UBSan: a random-operation driver (tests/native/bm_fuzz.cpp)
 built with g++ against the library's own block_manager.cpp checks the index
 against std::multimap under crowded keys, then the pool invariants after every
-operation.  No GPU."""
+operation, and every 250 operations the state image: restored into a fresh
+manager it gives the same state; corrupted (random words, truncations) it
+loads into a consistent state or changes nothing.  No GPU."""
 import os
 import shutil
 import subprocess
