@@ -1,13 +1,16 @@
 """Stateful property test of the host block manager against the oracle
 (hypothesis): random sequences of reservations, prompts with prefix reuse,
-registrations, forks, releases and matches -- edge cases included (empty
-prompts, zero-token registrations, full pools) -- with every status and the
-whole pool state compared bit-exact after each step.  No GPU."""
+registrations, forks, releases, matches and host state checkpoints (the
+state image saved and loaded into a fresh pool, which carries on) -- edge
+cases included (empty prompts, zero-token registrations, full pools) -- with
+every status and the whole pool state compared bit-exact after each step.
+No GPU."""
 import hypothesis.strategies as st
 import pytest
 from hypothesis import HealthCheck, settings
 from hypothesis.stateful import RuleBasedStateMachine, initialize, invariant, rule
 
+import pagedattention_decode_03_b200 as pa
 from oracle import Status
 
 from test_host_prefix import Both
@@ -57,6 +60,17 @@ class PoolMachine(RuleBasedStateMachine):
     @rule(toks=TOKENS)
     def match(self, toks):
         self.x.match(toks)
+
+    @rule()
+    def checkpoint(self):
+        """Carry on in a fresh pool restored from the state image."""
+        p = self.x.p
+        image = pa.pa_state_save(p)
+        fresh = pa.pa_pool_create(num_layers=1, num_kv_heads=1, block_size=p.block_size,
+                                  num_blocks=p.num_blocks, max_seqs=p.max_seqs,
+                                  max_blocks_per_seq=p.max_blocks_per_seq, host_only=True)
+        pa.pa_state_load(fresh, image)
+        self.x.p = fresh
 
     @invariant()
     def same(self):
