@@ -3,6 +3,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <utility>
 
 namespace pa {
 
@@ -501,8 +502,50 @@ Status BlockManager::load_state(const int32_t* w, size_t n) {
     const int kinds = (seen[b] ? 1 : 0) + (ref[b] > 0 ? 1 : 0) + (cached[b] ? 1 : 0);
     if (kinds != 1 || (cached[b] && bnode[b] < 0) || (seen[b] && bnode[b] >= 0)) return kInvalidArg;
   }
+  // the trie: a live node's parent is live, its child count is the live
+  // nodes naming it, it holds a block or leads to one, and its key is the
+  // hash of (parent, tokens)
+  std::vector<int32_t> kids(nn, 0);
+  for (int32_t c = 0; c < nn; ++c) {
+    if (dead[c]) continue;
+    const Node& nd = nodes[c];
+    if (nd.block >= 0 && bnode[nd.block] != c) return kInvalidArg;
+    if (nd.parent >= 0) {
+      if (dead[nd.parent]) return kInvalidArg;
+      ++kids[nd.parent];
+    }
+    if (nd.key != node_key(nd.parent, &toks[static_cast<size_t>(c) * block_size_])) return kInvalidArg;
+  }
   for (int32_t c = 0; c < nn; ++c)
-    if (!dead[c] && nodes[c].block >= 0 && bnode[nodes[c].block] != c) return kInvalidArg;
+    if (!dead[c] && (nodes[c].children != kids[c] || (nodes[c].block < 0 && kids[c] == 0)))
+      return kInvalidArg;
+  // every parent chain reaches the root (no cycle), and no two live nodes
+  // hold the same (parent, tokens)
+  std::vector<char> state(nn, 0);  // 0 unvisited, 1 on the current chain, 2 reaches the root
+  std::vector<int32_t> chain;
+  for (int32_t c = 0; c < nn; ++c) {
+    if (dead[c] || state[c] == 2) continue;
+    chain.clear();
+    int32_t v = c;
+    while (v >= 0 && state[v] == 0) {
+      state[v] = 1;
+      chain.push_back(v);
+      v = nodes[v].parent;
+    }
+    if (v >= 0 && state[v] == 1) return kInvalidArg;
+    for (int32_t u : chain) state[u] = 2;
+  }
+  NodeIndex idx;
+  for (int32_t c = 0; c < nn; ++c) {
+    if (dead[c]) continue;
+    const int32_t* tc = &toks[static_cast<size_t>(c) * block_size_];
+    const int32_t twin = idx.find(nodes[c].key, [&](int32_t o) {
+      return nodes[o].parent == nodes[c].parent &&
+             std::memcmp(&toks[static_cast<size_t>(o) * block_size_], tc, sizeof(int32_t) * block_size_) == 0;
+    });
+    if (twin >= 0) return kInvalidArg;
+    idx.insert(nodes[c].key, c);
+  }
 
   // apply
   std::fill(ring_.begin(), ring_.end(), 0);
@@ -515,9 +558,7 @@ Status BlockManager::load_state(const int32_t* w, size_t n) {
   nodes_.swap(nodes);
   node_tokens_.swap(toks);
   spare_nodes_.swap(spare);
-  index_ = NodeIndex();
-  for (int32_t c = 0; c < nn; ++c)
-    if (!dead[c]) index_.insert(nodes_[c].key, c);
+  index_ = std::move(idx);
   std::fill(lru_prev_.begin(), lru_prev_.end(), -2);
   std::fill(lru_next_.begin(), lru_next_.end(), -2);
   lru_head_ = lru_tail_ = -1;

@@ -83,6 +83,22 @@ def snapshot(p):
     return (pa.pa_get_free_list(p), pa.pa_get_cached_blocks(p), pa.pa_get_refcounts(p), tables)
 
 
+def trie_of(words):
+    """Offset of the node records in a state image, their count and the live
+    (not spare) nodes, following the image layout of block_manager.cpp."""
+    nb, B, max_seqs = words[1], words[2], words[3]
+    at = 5
+    at += 1 + words[at]                  # free list
+    at += 2 * nb                         # reference counts, block -> node
+    for _ in range(max_seqs):
+        at += 3 + words[at + 2]          # active, len, table size, table
+    nn = words[at]
+    nodes_at = at + 1
+    at = nodes_at + 5 * nn + nn * B
+    spare = set(words[at + 1: at + 1 + words[at]])
+    return nodes_at, nn, [c for c in range(nn) if c not in spare]
+
+
 @pytest.mark.parametrize("seed,nb,B", [(0, 40, 16), (1, 24, 16), (2, 48, 32), (3, 20, 16)])
 def test_restore_replays_exactly(seed, nb, B):
     vocab = 7
@@ -143,6 +159,15 @@ def test_refused_images_change_nothing():
     bad = list(words)
     bad[ref0 + nb] = nb + 7                              # a block names a node that does not exist
     refused(packed(bad))
+    # the prefix trie inside the image: a live node's child count, a parent
+    # cycle and a key that is not the hash of (parent, tokens)
+    nodes_at, nn, live = trie_of(words)
+    assert live, "the drive registered no prefix"
+    c = live[0]
+    for field, value in ((2, words[nodes_at + 5 * c + 2] + 1), (0, c), (3, words[nodes_at + 5 * c + 3] ^ 1)):
+        bad = list(words)
+        bad[nodes_at + 5 * c + field] = value
+        refused(packed(bad))
     other = Both(33, B)                                  # another geometry
     with pytest.raises(pa.PAError) as e:
         pa.pa_state_load(other.p, image)
