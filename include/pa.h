@@ -339,9 +339,11 @@ pa_status pa_state_size(const pa_pool *pool, size_t *bytes);
 pa_status pa_state_save(const pa_pool *pool, void *buf, size_t cap, size_t *written);
 
 /* Replace the pool's host state by the image in buf.  The whole image is
- * validated first: geometry, every id in range, and a consistent pool (each
+ * validated first: geometry, every id in range, a consistent pool (each
  * block exactly one of free, referenced by the tables it appears in, or idle
- * and cached; reference counts equal to those appearances).
+ * and cached; reference counts equal to those appearances) and a consistent
+ * prefix index (parent chains reach the root, child counts and keys match,
+ * no prefix twice, no node that holds no block and leads to none).
  * Errors: PA_ERR_INVALID_ARG (null argument, a truncated, corrupt or
  * inconsistent image, another geometry); on error nothing changes. */
 pa_status pa_state_load(pa_pool *pool, const void *buf, size_t bytes);
