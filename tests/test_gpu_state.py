@@ -15,6 +15,7 @@ import torch
 
 import pagedattention_decode_03_b200 as pa
 from paged_harness import Pair, from_dev, to_dev
+from test_gpu_siblings import family_workload
 from workloads import step_kv_bits, step_q_bits, workload
 
 pytestmark = pytest.mark.gpu
@@ -34,9 +35,15 @@ def twin(p):
     return b
 
 
-@pytest.mark.parametrize("name", ["tiny", "mha7b_share"])
+def case(name):
+    if name == "fp8_family":   # FP8 scales carried over; forks, sibling sets, a lone sequence
+        return family_workload(4, "fp8_e4m3", [(203, 3)], [300], steps=2)
+    return workload(name, steps=2)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mha7b_share", "fp8_family"])
 def test_restored_pool_decodes_like_the_saved_one(name):
-    w = workload(name, steps=2)
+    w = case(name)
     layers = [0] if w.num_layers > 1 else None
     p = Pair(w, layers=layers) if layers else Pair(w)
     if layers:
